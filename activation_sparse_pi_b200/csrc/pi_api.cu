@@ -1,0 +1,647 @@
+// C ABI of the predictor-gated sparse FFN (declared in include/pi.h).
+//
+// Host side: argument validation, workspace layout, kernel selection and
+// launches.  Every kernel is launched with programmatic stream serialization
+// so its prologue (barrier set-up, weight prefetch) overlaps the tail of the
+// kernel before it; each kernel waits (griddepcontrol.wait) before it touches
+// that kernel's results.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <set>
+#include <utility>
+#include <cstring>
+#include <string>
+
+#include "../../include/pi.h"
+#include "pi_generic.cuh"
+
+using namespace pi;
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_launches{0};
+
+int32_t fail(int32_t status, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int32_t fail(int32_t status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+
+#define PI_CUDA(call)                                                                    \
+  do {                                                                                   \
+    cudaError_t e_ = (call);                                                             \
+    if (e_ != cudaSuccess)                                                               \
+      return fail(PI_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));          \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+  static thread_local int cached_dev = -1, cached = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev != cached_dev) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cached = v;
+    cached_dev = dev;
+  }
+  return cached;
+}
+
+constexpr size_t kSmemMax = 227 * 1024;
+constexpr size_t kSmemPred1 = 96 * 1024;
+constexpr size_t kSmemPred2 = 160 * 1024;
+constexpr size_t kSmemFfn = 180 * 1024;
+constexpr size_t kPartCap = 64ull << 20;  // bytes of batched down partials
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ------------------------------------------------------------ workspace
+struct WsLayout {
+  size_t a, mask, idx, count, xl, part, h, total;
+};
+
+int down_slices(int d, int B, int nsm) {
+  const int ndc = (d / 8 + 255) / 256;
+  int S = std::max(1, 2 * nsm / ndc);
+  const size_t per = (size_t)B * d * 4;
+  S = (int)std::min<size_t>((size_t)S, std::max<size_t>(1, kPartCap / per));
+  return S;
+}
+
+WsLayout ws_layout(int d, int F, int r, int B) {
+  const int nsm = num_sms();
+  WsLayout w{};
+  size_t o = 0;
+  w.a = o;     o += al256((size_t)B * r * 4);
+  w.mask = o;  o += al256((size_t)B * (F / 32) * 4);
+  w.idx = o;   o += al256((size_t)F * 4);
+  w.count = o; o += 256;
+  w.xl = o;    o += al256((size_t)B * d * 2);
+  const int G = std::max(nsm, down_slices(d, B, nsm));
+  w.part = o;  o += al256((size_t)G * B * d * 4);
+  w.h = o;     o += al256((size_t)F * B * 4);
+  w.total = o;
+  return w;
+}
+
+// ------------------------------------------------------------ launching
+template <typename Kern, typename... Args>
+cudaError_t launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args... args) {
+  if (smem > 48 * 1024) {
+    // once per (device, kernel): allow the large dynamic shared memory carve-out
+    static std::mutex mu;
+    static std::set<std::pair<int, const void*>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const auto key = std::make_pair(dev, reinterpret_cast<const void*>(kern));
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done.count(key)) {
+      e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax);
+      if (e != cudaSuccess) return e;
+      done.insert(key);
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
+// ------------------------------------------------------------ validation
+int check_act_dtype(int dt) { return dt == PI_F16 || dt == PI_BF16; }
+
+int32_t validate_predictor(const pi_predictor* p) {
+  if (!p) return fail(PI_ERR_INVALID_ARG, "predictor is NULL");
+  if (!check_act_dtype(p->dtype))
+    return fail(PI_ERR_UNSUPPORTED, "predictor dtype must be PI_F16 or PI_BF16 (got %d)", p->dtype);
+  if (p->d_model < 32 || p->d_model > 8192 || p->d_model % 32)
+    return fail(PI_ERR_UNSUPPORTED, "d_model %d: need 32 <= d_model <= 8192, multiple of 32",
+                p->d_model);
+  if (p->d_ff < 32 || p->d_ff > 65536 || p->d_ff % 32)
+    return fail(PI_ERR_UNSUPPORTED, "d_ff %d: need 32 <= d_ff <= 65536, multiple of 32", p->d_ff);
+  if (p->rank < 8 || p->rank > 2048 || p->rank % 8)
+    return fail(PI_ERR_UNSUPPORTED, "rank %d: need 8 <= rank <= 2048, multiple of 8", p->rank);
+  if (!p->w1 || !p->w2 || !p->b2) return fail(PI_ERR_INVALID_ARG, "predictor w1, w2 and b2 are required");
+  if (!aligned16(p->w1) || !aligned16(p->w2) || !aligned16(p->b2) || (p->b1 && !aligned16(p->b1)))
+    return fail(PI_ERR_INVALID_ARG, "predictor pointers must be 16-byte aligned");
+  return PI_OK;
+}
+
+int32_t validate_layer(const pi_layer* L) {
+  if (!L) return fail(PI_ERR_INVALID_ARG, "layer is NULL");
+  if (int32_t s = validate_predictor(&L->pred)) return s;
+  if (L->d_model != L->pred.d_model || L->d_ff != L->pred.d_ff)
+    return fail(PI_ERR_INVALID_ARG, "layer and predictor disagree on d_model/d_ff");
+  if (!check_act_dtype(L->adtype) || L->adtype != L->pred.dtype)
+    return fail(PI_ERR_UNSUPPORTED, "adtype must be PI_F16/PI_BF16 and equal the predictor dtype");
+  if (L->act != PI_RELU && L->act != PI_REGLU)
+    return fail(PI_ERR_UNSUPPORTED, "act must be PI_RELU or PI_REGLU");
+  if (L->wdtype == PI_F16 || L->wdtype == PI_BF16) {
+    if (L->wdtype != L->adtype)
+      return fail(PI_ERR_UNSUPPORTED, "16-bit weights must have the activation dtype");
+  } else if (L->wdtype == PI_Q4_0) {
+    if (L->adtype != PI_F16) return fail(PI_ERR_UNSUPPORTED, "Q4_0 weights need fp16 activations");
+    if (L->d_model % 256)
+      return fail(PI_ERR_UNSUPPORTED, "Q4_0 needs d_model %% 256 == 0 (16-byte aligned rows)");
+  } else {
+    return fail(PI_ERR_UNSUPPORTED, "wdtype %d unknown", L->wdtype);
+  }
+  if (!L->w_up || !L->w_down_t) return fail(PI_ERR_INVALID_ARG, "w_up and w_down_t are required");
+  if ((L->act == PI_REGLU) != (L->w_gate != nullptr))
+    return fail(PI_ERR_INVALID_ARG, "w_gate must be given exactly for ReGLU");
+  if (L->act == PI_RELU && L->b_gate)
+    return fail(PI_ERR_INVALID_ARG, "b_gate is only meaningful for ReGLU");
+  if (L->act == PI_REGLU && L->b_up)
+    return fail(PI_ERR_INVALID_ARG, "ReGLU has no up-projection bias (use b_gate)");
+  const void* ps[] = {L->w_up, L->w_gate, L->w_down_t, L->b_up, L->b_gate};
+  for (const void* q : ps)
+    if (q && !aligned16(q)) return fail(PI_ERR_INVALID_ARG, "layer pointers must be 16-byte aligned");
+  return PI_OK;
+}
+
+int32_t validate_batch(int B) {
+  if (B < 1 || B > kMaxBatch)
+    return fail(PI_ERR_UNSUPPORTED, "batch %d: need 1 <= batch <= %d", B, kMaxBatch);
+  return PI_OK;
+}
+
+int32_t check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return PI_OK;
+  if (!ws) return fail(PI_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
+  if (!aligned16(ws)) return fail(PI_ERR_WORKSPACE, "workspace must be 16-byte aligned");
+  if (have < need) return fail(PI_ERR_WORKSPACE, "workspace has %zu bytes, need %zu", have, need);
+  return PI_OK;
+}
+
+// ------------------------------------------------------------ predictor
+template <int DT, int B, int CPT>
+cudaError_t launch_pred1(const pi_predictor* P, const uint16_t* x, const float* xr,
+                         uint16_t* xo, float* a, cudaStream_t st) {
+  const int nsm = num_sms();
+  Pred1Params p{};
+  p.w1 = static_cast<const uint8_t*>(P->w1);
+  p.b1 = P->b1;
+  p.x = x;
+  p.x_resid = xr;
+  p.x_out = xo;
+  p.a = a;
+  p.d = P->d_model;
+  p.r = P->rank;
+  const int G = std::min(nsm, P->rank);
+  p.rows_per_cta = (P->rank + G - 1) / G;
+  const size_t row = (size_t)P->d_model * 2;
+  const size_t xb = ((size_t)B * P->d_model * 2 + 127) & ~size_t(127);
+  const size_t avail = kSmemPred1 > 2048 + xb ? kSmemPred1 - 2048 - xb : 0;
+  p.nstages = (int)std::max<size_t>(kRowGroup, std::min<size_t>(std::max(p.rows_per_cta, kRowGroup),
+                                                                std::min<size_t>(32, avail / row)));
+  const size_t smem = 2048 + xb + (size_t)p.nstages * row;
+  return launch(k_pred1<DT, B, CPT>, dim3(G), dim3(kThreads), smem, st, p);
+}
+
+// x held in registers: B x CPT 16-byte chunks per thread (B * CPT <= 16)
+bool pred1_fused_ok(int B, int d) {
+  const int cpt = (d / 8 + kConsumers - 1) / kConsumers;
+  return (B == 1 || B == 2 || B == 4) && cpt <= 4 && B * cpt <= 8;
+}
+
+template <int DT, int B>
+cudaError_t pred1_cpt(const pi_predictor* P, const uint16_t* x, const float* xr, uint16_t* xo,
+                      float* a, cudaStream_t st) {
+  const int cpt = (P->d_model / 8 + kConsumers - 1) / kConsumers;
+  if (cpt <= 1) return launch_pred1<DT, B, 1>(P, x, xr, xo, a, st);
+  if (cpt <= 2) return launch_pred1<DT, B, 2>(P, x, xr, xo, a, st);
+  if constexpr (B <= 2) return launch_pred1<DT, B, 4>(P, x, xr, xo, a, st);
+  return cudaErrorInvalidValue;
+}
+
+template <int DT>
+cudaError_t pred1_dispatch(const pi_predictor* P, int B, const uint16_t* x, const float* xr,
+                           uint16_t* xo, float* a, cudaStream_t st) {
+  switch (B) {
+    case 1: return pred1_cpt<DT, 1>(P, x, xr, xo, a, st);
+    case 2: return pred1_cpt<DT, 2>(P, x, xr, xo, a, st);
+    default: return pred1_cpt<DT, 4>(P, x, xr, xo, a, st);
+  }
+}
+
+int cpl_for(int r) {
+  const int need = (r / 8 + 31) / 32;
+  for (int c : {1, 2, 4, 6, 8})
+    if (c >= need) return c;
+  return 0;
+}
+
+bool pred2_fused_ok(int B, int r) {
+  const int c = cpl_for(r);
+  return c > 0 && (B == 1 || B == 2) && B * c <= 8;
+}
+
+template <int DT, int B, int CPL>
+cudaError_t launch_pred2(const pi_predictor* P, const float* a, uint32_t* mask, float* logits,
+                         cudaStream_t st) {
+  const int nsm = num_sms();
+  Pred2Params p{};
+  p.w2 = static_cast<const uint8_t*>(P->w2);
+  p.b2 = P->b2;
+  p.a = a;
+  p.mask = mask;
+  p.logits = logits;
+  p.threshold = P->threshold;
+  p.F = P->d_ff;
+  p.r = P->rank;
+  const int nunits = P->d_ff / 32;
+  p.units_per_cta = (nunits + nsm - 1) / nsm;
+  const int G = (nunits + p.units_per_cta - 1) / p.units_per_cta;
+  const size_t stage = (size_t)8 * P->rank * 2;
+  const size_t fixed = 1024 + (((size_t)p.units_per_cta * 32 * 4 + 127) & ~size_t(127));
+  const size_t avail = kSmemPred2 > fixed ? kSmemPred2 - fixed : 0;
+  // a unit's four stages go to four warp pairs; with fewer than four stages a
+  // pair could wait on a stage phase ahead of the one in progress
+  p.nstages = (int)std::min<size_t>((size_t)4 * p.units_per_cta, std::min<size_t>(32, avail / stage));
+  if (p.nstages < 4 && p.nstages < 4 * p.units_per_cta) return cudaErrorInvalidValue;
+  const size_t smem = fixed + (size_t)p.nstages * stage;
+  return launch(k_pred2<DT, B, CPL>, dim3(G), dim3(kThreads), smem, st, p);
+}
+
+template <int DT, int B>
+cudaError_t pred2_cpl(const pi_predictor* P, const float* a, uint32_t* mask, float* logits,
+                      cudaStream_t st) {
+  switch (cpl_for(P->rank)) {
+    case 1: return launch_pred2<DT, B, 1>(P, a, mask, logits, st);
+    case 2: return launch_pred2<DT, B, 2>(P, a, mask, logits, st);
+    case 4: return launch_pred2<DT, B, 4>(P, a, mask, logits, st);
+    case 6: if constexpr (B == 1) return launch_pred2<DT, B, 6>(P, a, mask, logits, st); break;
+    case 8: if constexpr (B == 1) return launch_pred2<DT, B, 8>(P, a, mask, logits, st); break;
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int DT, int MODE, int BB>
+cudaError_t launch_rows(const RowsParams& p, int nrows_work, cudaStream_t st) {
+  const int nsm = num_sms();
+  const int warps = std::max(1, nrows_work);
+  const int blocks = std::min((warps + 7) / 8, nsm * 8);
+  return launch(k_rows<MODE, DT, 0, BB>, dim3(blocks), dim3(256), 0, st, p);
+}
+
+template <int DT, int MODE>
+cudaError_t rows_bb(const RowsParams& p, int nrows_work, cudaStream_t st) {
+  if (p.B <= 8) return launch_rows<DT, MODE, 8>(p, nrows_work, st);
+  if (p.B <= 32) return launch_rows<DT, MODE, 32>(p, nrows_work, st);
+  return launch_rows<DT, MODE, 64>(p, nrows_work, st);
+}
+
+// x16: 16-bit input, or null with xr (residual) given; xo receives x_l then.
+template <int DT>
+int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const float* xr,
+                     uint16_t* xo, uint32_t* mask, float* logits, float* a, cudaStream_t st) {
+  const int d = P->d_model;
+  if (pred1_fused_ok(B, d)) {
+    PI_CUDA((pred1_dispatch<DT>(P, B, x16, xr, xo, a, st)));
+  } else {
+    if (xr) {
+      PI_CUDA((launch(k_cast_rms<DT>, dim3(B), dim3(256), 0, st, xr, xo, d)));
+      x16 = xo;
+    }
+    RowsParams p{};
+    p.w = static_cast<const uint8_t*>(P->w1);
+    p.bias = P->b1;
+    p.x16 = x16;
+    p.out = a;
+    p.nrows = P->rank;
+    p.len = d;
+    p.B = B;
+    PI_CUDA((rows_bb<DT, kModePred1>(p, P->rank, st)));
+  }
+  if (pred2_fused_ok(B, P->rank)) {
+    if (B == 1) PI_CUDA((pred2_cpl<DT, 1>(P, a, mask, logits, st)));
+    else PI_CUDA((pred2_cpl<DT, 2>(P, a, mask, logits, st)));
+  } else {
+    PI_CUDA(cudaMemsetAsync(mask, 0, (size_t)B * (P->d_ff / 32) * 4, st));
+    RowsParams p{};
+    p.w = static_cast<const uint8_t*>(P->w2);
+    p.bias = P->b2;
+    p.x32 = a;
+    p.out = logits;
+    p.mask = mask;
+    p.threshold = P->threshold;
+    p.nrows = P->d_ff;
+    p.len = P->rank;
+    p.B = B;
+    PI_CUDA((rows_bb<DT, kModePred2>(p, P->d_ff, st)));
+  }
+  return PI_OK;
+}
+
+// ------------------------------------------------------------ gathered FFN
+int cpt_for(int wdt, int d) {
+  const int units = wdt == PI_Q4_0 ? d / 32 : d / 8;
+  const int need = (units + kConsumers - 1) / kConsumers;
+  for (int c : {1, 2, 4})
+    if (c >= need) return c;
+  return 0;
+}
+
+int ffn_nstages(const pi_layer* L) {
+  const size_t rb = L->wdtype == PI_Q4_0 ? (size_t)L->d_model / 32 * 18 : (size_t)L->d_model * 2;
+  const size_t stage = rb * (L->act == PI_REGLU ? 3 : 2);
+  const size_t fixed = 1024 + 4096;
+  return (int)std::min<size_t>(32, (kSmemFfn - fixed) / stage);
+}
+
+bool ffn_fused_ok(const pi_layer* L, int B) {
+  if (!(B == 1 || B == 2 || B == 4)) return false;
+  const int c = cpt_for(L->wdtype, L->d_model);
+  if (c == 0) return false;
+  if (L->wdtype == PI_Q4_0 ? (B * c > 2) : (B * c > 8)) return false;
+  return ffn_nstages(L) >= kGroup;
+}
+
+template <int WDT, int ACT, int B, int CPT>
+cudaError_t launch_ffn(const pi_layer* L, const uint16_t* x, const int32_t* idx,
+                       const int32_t* count, float* part, cudaStream_t st) {
+  FfnParams p{};
+  p.w_act = static_cast<const uint8_t*>(ACT == 1 ? L->w_gate : L->w_up);
+  p.w_up = static_cast<const uint8_t*>(L->w_up);
+  p.w_dn = static_cast<const uint8_t*>(L->w_down_t);
+  p.b_act = ACT == 1 ? L->b_gate : L->b_up;
+  p.x = x;
+  p.idx = idx;
+  p.count = count;
+  p.part = part;
+  p.d = L->d_model;
+  p.F = L->d_ff;
+  p.row_bytes = WDT == 2 ? (uint32_t)(L->d_model / 32 * 18) : (uint32_t)(L->d_model * 2);
+  p.nstages = ffn_nstages(L);
+  const size_t smem = 1024 + 4096 + (size_t)p.nstages * p.row_bytes * (ACT == 1 ? 3 : 2);
+  return launch(k_ffn<WDT, ACT, B, CPT>, dim3(num_sms()), dim3(kThreads), smem, st, p);
+}
+
+template <int WDT, int ACT, int B>
+cudaError_t ffn_cpt(const pi_layer* L, const uint16_t* x, const int32_t* idx, const int32_t* count,
+                    float* part, cudaStream_t st) {
+  const int c = cpt_for(L->wdtype, L->d_model);
+  if constexpr (WDT == 2) {
+    if (c == 1) return launch_ffn<WDT, ACT, B, 1>(L, x, idx, count, part, st);
+  } else {
+    if (c == 1) return launch_ffn<WDT, ACT, B, 1>(L, x, idx, count, part, st);
+    if (c == 2 && B <= 4) return launch_ffn<WDT, ACT, B, 2>(L, x, idx, count, part, st);
+    if constexpr (B <= 2)
+      if (c == 4) return launch_ffn<WDT, ACT, B, 4>(L, x, idx, count, part, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int WDT, int ACT>
+cudaError_t ffn_b(const pi_layer* L, int B, const uint16_t* x, const int32_t* idx,
+                  const int32_t* count, float* part, cudaStream_t st) {
+  if (B == 1) return ffn_cpt<WDT, ACT, 1>(L, x, idx, count, part, st);
+  if (B == 2) return ffn_cpt<WDT, ACT, 2>(L, x, idx, count, part, st);
+  if constexpr (WDT != 2) return ffn_cpt<WDT, ACT, 4>(L, x, idx, count, part, st);
+  return cudaErrorInvalidValue;
+}
+
+template <int WDT, int ACT>
+cudaError_t launch_up_generic(const pi_layer* L, int B, const uint16_t* x, const int32_t* idx,
+                              const int32_t* count, float* h, cudaStream_t st) {
+  RowsParams p{};
+  p.w = static_cast<const uint8_t*>(ACT == 1 ? L->w_gate : L->w_up);
+  p.w2nd = static_cast<const uint8_t*>(L->w_up);
+  p.bias = ACT == 1 ? L->b_gate : L->b_up;
+  p.x16 = x;
+  p.idx = idx;
+  p.count = count;
+  p.out = h;
+  p.nrows = L->d_ff;
+  p.len = L->d_model;
+  p.B = B;
+  const int nsm = num_sms();
+  const int blocks = std::min((L->d_ff + 7) / 8, nsm * 8);
+  if (B <= 8) return launch(k_rows<kModeUp, WDT, ACT, 8>, dim3(blocks), dim3(256), 0, st, p);
+  if (B <= 32) return launch(k_rows<kModeUp, WDT, ACT, 32>, dim3(blocks), dim3(256), 0, st, p);
+  return launch(k_rows<kModeUp, WDT, ACT, 64>, dim3(blocks), dim3(256), 0, st, p);
+}
+
+// mode 0: y = FFN(x); mode 1: out += FFN(x).  ev (optional): two events recorded
+// right before and right after the gathered-FFN kernel.
+int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const int32_t* idx,
+                 const int32_t* count, float* out, int mode, const WsLayout& w, uint8_t* ws,
+                 cudaStream_t st, void* const* ev = nullptr) {
+  if (ev) PI_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(ev[0]), st));
+  float* part = reinterpret_cast<float*>(ws + w.part);
+  const int d = L->d_model;
+  const int n4 = B * d / 4;
+  int G;
+  if (ffn_fused_ok(L, B)) {
+    cudaError_t e = cudaErrorInvalidValue;
+    const int act = L->act;
+    switch (L->wdtype) {
+      case PI_F16: e = act ? ffn_b<0, 1>(L, B, x, idx, count, part, st) : ffn_b<0, 0>(L, B, x, idx, count, part, st); break;
+      case PI_BF16: e = act ? ffn_b<1, 1>(L, B, x, idx, count, part, st) : ffn_b<1, 0>(L, B, x, idx, count, part, st); break;
+      case PI_Q4_0: e = act ? ffn_b<2, 1>(L, B, x, idx, count, part, st) : ffn_b<2, 0>(L, B, x, idx, count, part, st); break;
+    }
+    if (e != cudaSuccess) return fail(PI_ERR_CUDA, "fused FFN launch failed: %s", cudaGetErrorString(e));
+    G = num_sms();
+  } else {
+    float* h = reinterpret_cast<float*>(ws + w.h);
+    cudaError_t e = cudaErrorInvalidValue;
+    const int act = L->act;
+    switch (L->wdtype) {
+      case PI_F16: e = act ? launch_up_generic<0, 1>(L, B, x, idx, count, h, st) : launch_up_generic<0, 0>(L, B, x, idx, count, h, st); break;
+      case PI_BF16: e = act ? launch_up_generic<1, 1>(L, B, x, idx, count, h, st) : launch_up_generic<1, 0>(L, B, x, idx, count, h, st); break;
+      case PI_Q4_0: e = act ? launch_up_generic<2, 1>(L, B, x, idx, count, h, st) : launch_up_generic<2, 0>(L, B, x, idx, count, h, st); break;
+    }
+    if (e != cudaSuccess) return fail(PI_ERR_CUDA, "batched up launch failed: %s", cudaGetErrorString(e));
+    DownParams dp{};
+    dp.w_dn = static_cast<const uint8_t*>(L->w_down_t);
+    dp.idx = idx;
+    dp.count = count;
+    dp.h = h;
+    dp.part = part;
+    dp.d = d;
+    dp.F = L->d_ff;
+    dp.B = B;
+    G = down_slices(d, B, num_sms());
+    dim3 grid((d / 8 + 255) / 256, G);
+    switch (L->wdtype) {
+      case PI_F16: e = launch(k_down<0>, grid, dim3(256), 0, st, dp); break;
+      case PI_BF16: e = launch(k_down<1>, grid, dim3(256), 0, st, dp); break;
+      default: e = launch(k_down<2>, grid, dim3(256), 0, st, dp); break;
+    }
+    if (e != cudaSuccess) return fail(PI_ERR_CUDA, "batched down launch failed: %s", cudaGetErrorString(e));
+  }
+  if (ev) PI_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(ev[1]), st));
+  const dim3 rg((n4 + 31) / 32);
+  if (mode == 0) PI_CUDA((launch(k_reduce<0>, rg, dim3(256), 0, st, (const float*)part, G, n4, out)));
+  else PI_CUDA((launch(k_reduce<1>, rg, dim3(256), 0, st, (const float*)part, G, n4, out)));
+  return PI_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* pi_status_string(int32_t s) {
+  switch (s) {
+    case PI_OK: return "success";
+    case PI_ERR_INVALID_ARG: return "invalid argument";
+    case PI_ERR_UNSUPPORTED: return "unsupported shape, dtype or batch";
+    case PI_ERR_WORKSPACE: return "workspace missing or too small";
+    case PI_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+  }
+}
+
+const char* pi_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t pi_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int32_t pi_device_error(int32_t* code_out) {
+  if (!code_out) return fail(PI_ERR_INVALID_ARG, "code_out is NULL");
+  PI_CUDA(cudaDeviceSynchronize());
+  int v = 0;
+  PI_CUDA(cudaMemcpyFromSymbol(&v, g_dev_error, sizeof v));
+  const int zero = 0;
+  PI_CUDA(cudaMemcpyToSymbol(g_dev_error, &zero, sizeof zero));
+  *code_out = v;
+  return PI_OK;
+}
+
+size_t pi_workspace_size(const pi_layer* layers, int32_t n_layers, int32_t batch) {
+  if (!layers || n_layers < 1 || validate_batch(batch)) return 0;
+  int d = 0, F = 0, r = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    if (validate_layer(&layers[l])) return 0;
+    d = std::max(d, layers[l].d_model);
+    F = std::max(F, layers[l].d_ff);
+    r = std::max(r, layers[l].pred.rank);
+  }
+  return ws_layout(d, F, r, batch).total;
+}
+
+int32_t pi_predict(const pi_predictor* pred, const void* x, int32_t batch, uint32_t* mask_bits,
+                   float* logits, void* workspace, size_t workspace_bytes, void* stream) {
+  if (int32_t s = validate_predictor(pred)) return s;
+  if (int32_t s = validate_batch(batch)) return s;
+  if (!x || !mask_bits) return fail(PI_ERR_INVALID_ARG, "x and mask_bits are required");
+  if (!aligned16(x) || !aligned16(mask_bits) || (logits && !aligned16(logits)))
+    return fail(PI_ERR_INVALID_ARG, "x, mask_bits and logits must be 16-byte aligned");
+  const WsLayout w = ws_layout(pred->d_model, pred->d_ff, pred->rank, batch);
+  if (int32_t s = check_ws(workspace, workspace_bytes, w.a + (size_t)batch * pred->rank * 4)) return s;
+  float* a = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint16_t* x16 = static_cast<const uint16_t*>(x);
+  if (pred->dtype == PI_F16)
+    return predict_impl<0>(pred, batch, x16, nullptr, nullptr, mask_bits, logits, a, st);
+  return predict_impl<1>(pred, batch, x16, nullptr, nullptr, mask_bits, logits, a, st);
+}
+
+int32_t pi_compact(const uint32_t* mask_bits, int32_t batch, int32_t d_ff, int32_t* idx,
+                   int32_t* count, void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (int32_t s = validate_batch(batch)) return s;
+  if (d_ff < 32 || d_ff > 65536 || d_ff % 32)
+    return fail(PI_ERR_UNSUPPORTED, "d_ff %d: need 32 <= d_ff <= 65536, multiple of 32", d_ff);
+  if (!mask_bits || !idx || !count) return fail(PI_ERR_INVALID_ARG, "mask_bits, idx and count are required");
+  if (!aligned16(mask_bits) || !aligned16(idx) || (reinterpret_cast<uintptr_t>(count) & 3u))
+    return fail(PI_ERR_INVALID_ARG, "mask_bits and idx must be 16-byte aligned, count 4-byte aligned");
+  PI_CUDA((launch(k_compact, dim3(1), dim3(kCompactThreads), 0, static_cast<cudaStream_t>(stream),
+                  mask_bits, (int)batch, (int)d_ff, idx, count)));
+  return PI_OK;
+}
+
+int32_t pi_sparse_ffn(const pi_layer* layer, const void* x, int32_t batch, const int32_t* idx,
+                      const int32_t* count, float* y, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  if (int32_t s = validate_layer(layer)) return s;
+  if (int32_t s = validate_batch(batch)) return s;
+  if (!x || !idx || !count || !y) return fail(PI_ERR_INVALID_ARG, "x, idx, count and y are required");
+  if (!aligned16(x) || !aligned16(idx) || !aligned16(y) || (reinterpret_cast<uintptr_t>(count) & 3u))
+    return fail(PI_ERR_INVALID_ARG, "x, idx and y must be 16-byte aligned, count 4-byte aligned");
+  const WsLayout w = ws_layout(layer->d_model, layer->d_ff, layer->pred.rank, batch);
+  if (int32_t s = check_ws(workspace, workspace_bytes, w.total)) return s;
+  return ffn_impl(layer, batch, static_cast<const uint16_t*>(x), idx, count, y, 0, w,
+                  static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+int32_t pi_ffn_stack(const pi_layer* layers, int32_t n_layers, float* x_resid, int32_t batch,
+                     int32_t* idx_out, int32_t* count_out, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  return pi_ffn_stack_timed(layers, n_layers, x_resid, batch, idx_out, count_out, workspace,
+                            workspace_bytes, stream, nullptr);
+}
+
+int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_resid,
+                           int32_t batch, int32_t* idx_out, int32_t* count_out, void* workspace,
+                           size_t workspace_bytes, void* stream, void* const* ffn_events) {
+  if (!layers || n_layers < 1) return fail(PI_ERR_INVALID_ARG, "need at least one layer");
+  if (int32_t s = validate_batch(batch)) return s;
+  if (!x_resid || !aligned16(x_resid)) return fail(PI_ERR_INVALID_ARG, "x_resid must be a 16-byte aligned pointer");
+  if ((idx_out && !aligned16(idx_out)) || (count_out && (reinterpret_cast<uintptr_t>(count_out) & 3u)))
+    return fail(PI_ERR_INVALID_ARG, "idx_out must be 16-byte aligned, count_out 4-byte aligned");
+  int d = 0, F = 0, r = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    if (int32_t s = validate_layer(&layers[l])) return s;
+    if (layers[l].d_model != layers[0].d_model || layers[l].adtype != layers[0].adtype)
+      return fail(PI_ERR_INVALID_ARG, "all layers of a stack need the same d_model and adtype");
+    if (idx_out && layers[l].d_ff != layers[0].d_ff)
+      return fail(PI_ERR_INVALID_ARG, "idx_out needs the same d_ff in every layer");
+    d = std::max(d, layers[l].d_model);
+    F = std::max(F, layers[l].d_ff);
+    r = std::max(r, layers[l].pred.rank);
+  }
+  const WsLayout w = ws_layout(d, F, r, batch);
+  if (int32_t s = check_ws(workspace, workspace_bytes, w.total)) return s;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint16_t* xl = reinterpret_cast<uint16_t*>(ws + w.xl);
+  float* a = reinterpret_cast<float*>(ws + w.a);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(ws + w.mask);
+  for (int l = 0; l < n_layers; ++l) {
+    const pi_layer* L = &layers[l];
+    int32_t* idx = idx_out ? idx_out + (size_t)l * L->d_ff : reinterpret_cast<int32_t*>(ws + w.idx);
+    int32_t* cnt = count_out ? count_out + l : reinterpret_cast<int32_t*>(ws + w.count);
+    int32_t s = (L->adtype == PI_F16)
+                    ? predict_impl<0>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, st)
+                    : predict_impl<1>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, st);
+    if (s) return s;
+    PI_CUDA((launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, (const uint32_t*)mask,
+                    (int)batch, L->d_ff, idx, cnt)));
+    if (ffn_events && (!ffn_events[2 * l] || !ffn_events[2 * l + 1]))
+      return fail(PI_ERR_INVALID_ARG, "ffn_events[%d..%d] must be events", 2 * l, 2 * l + 1);
+    if ((s = ffn_impl(L, batch, xl, idx, cnt, x_resid, 1, w, ws, st,
+                      ffn_events ? ffn_events + 2 * l : nullptr)))
+      return s;
+  }
+  return PI_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,185 @@
+// Device helpers shared by the sparse-FFN kernels (sm_100a).
+//
+// Data movement uses the sm_90+/sm_100 bulk-copy engine (cp.async.bulk,
+// 1-D, global -> shared, completion counted on an mbarrier).  Every wait on
+// an mbarrier is bounded: after kWaitLimit polls the kernel records
+// kErrTimeout in the device error word and the caller bails out.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pi {
+
+constexpr int kMaxBatch = 64;
+constexpr int kErrTimeout = 1;
+constexpr int kErrBadIndex = 2;
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+// Device error word (read and cleared by pi_device_error()).
+__device__ int g_dev_error;
+
+__device__ __forceinline__ void set_error(int code) { atomicOr(&g_dev_error, code); }
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for the phase with the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kWaitLimit; ++it)
+    if (mbar_try_wait(bar, parity)) return true;
+  set_error(kErrTimeout);
+  return false;
+}
+
+// ------------------------------------------------------------- bulk copies
+// 1-D bulk copy global -> shared; dst, src 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// Same, with an L2 eviction-priority policy (streamed once: evict first).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
+      "%2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// ------------------------------------------- programmatic dependent launch
+// Wait until the preceding kernel in the stream has completed and its memory
+// is visible (no-op when the kernel was not launched as a dependent).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next kernel in the stream to start its prologue.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ----------------------------------------------------- 16-bit arithmetic
+// DT: 0 = fp16, 1 = bf16.  A 32-bit word holds two consecutive elements, the
+// lower-addressed one in the low half.
+template <int DT>
+__device__ __forceinline__ float2 unpack2(uint32_t u) {
+  if constexpr (DT == 0) {
+    __half2 h = *reinterpret_cast<__half2*>(&u);
+    return __half22float2(h);
+  } else {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+  }
+}
+
+// acc0 += w.lo * x.lo, acc1 += w.hi * x.hi with both operands 16-bit; the
+// products are exact and each accumulation is one fp32 rounding.
+template <int DT>
+__device__ __forceinline__ void dot2(uint32_t w, uint32_t x, float& acc0, float& acc1) {
+  if constexpr (DT == 0) {
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+        "mov.b32 {wl, wh}, %2;\n\tmov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, wl, xl, %0;\n\tfma.rn.f32.f16 %1, wh, xh, %1;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(w), "r"(x));
+  } else {
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+        "mov.b32 {wl, wh}, %2;\n\tmov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\tfma.rn.f32.bf16 %1, wh, xh, %1;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(w), "r"(x));
+  }
+}
+
+// Round an fp32 value to the 16-bit activation type (nearest even), as bits.
+template <int DT>
+__device__ __forceinline__ uint16_t round16(float v) {
+  if constexpr (DT == 0) {
+    return __half_as_ushort(__float2half_rn(v));
+  } else {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  }
+}
+
+// Q4_0 nibble q (0..15) -> (q - 8) as an exact fp32: place q in the low
+// mantissa bits of 2^23 and subtract 2^23 + 8.
+__device__ __forceinline__ float q4_val(uint32_t q) {
+  return __uint_as_float(0x4B000000u | q) - 8388616.0f;
+}
+
+// ------------------------------------------------------- warp reductions
+// Transposed reduction of V values (V a power of two, V <= 32) across the
+// warp.  Afterwards every lane holds the warp sum of value (lane >> (5 -
+// log2 V)) in v[0].
+template <int V>
+__device__ __forceinline__ float warp_reduce_transposed(float (&v)[V]) {
+  const int lane = threadIdx.x & 31;
+  int n = V;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    if (n > 1) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < V / 2; ++i) {
+        if (i < n / 2) {
+          float send = upper ? v[i] : v[i + n / 2];
+          float keep = upper ? v[i + n / 2] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      n >>= 1;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    }
+  }
+  return v[0];
+}
+
+template <int V>
+__device__ __forceinline__ constexpr int log2c() {
+  return V <= 1 ? 0 : 1 + log2c<V / 2>();
+}
+
+}  // namespace pi

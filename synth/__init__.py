@@ -11,6 +11,7 @@ from .layers import (
     LayerData,
     make_layer,
     make_tokens,
+    with_mode,
     zipf_profile,
     quantize_q4_0,
     q4_0_row_bytes,
@@ -23,6 +24,7 @@ __all__ = [
     "LayerData",
     "make_layer",
     "make_tokens",
+    "with_mode",
     "zipf_profile",
     "quantize_q4_0",
     "q4_0_row_bytes",

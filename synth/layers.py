@@ -128,7 +128,7 @@ def _bvn_cdf(h, k, rho):
     return 0.5 * (ndtr(h) + ndtr(k)) - owens_t(h, ah) - owens_t(k, ak) - beta
 
 
-def _bisect(f, target, lo, hi, iters=100):
+def _bisect(f, target, lo, hi, iters=60):
     """Root of the increasing function f(x) = target on [lo, hi]."""
     for _ in range(iters):
         mid = 0.5 * (lo + hi)
@@ -159,6 +159,9 @@ class LayerData:
     delta: float
     expected_pred_frac: float
     expected_recall: float
+    bias64: Optional[np.ndarray] = None   # [F] activation-row bias before rounding
+    deltas: Optional[dict] = None         # {"R": delta_R, "F": delta_F}
+    stats: Optional[dict] = None          # expected fraction / recall per mode
 
     def tensors(self):
         return {k: getattr(self, k) for k in
@@ -240,10 +243,10 @@ def make_layer(cfg: Config, layer: int, device="cpu", mode: str = "R") -> LayerD
         return float(_bvn_cdf(b / su, (b + delta) / sv, rho).sum() / p.sum())
 
     span = 20.0 * float(su.max() + sv.max())
-    if mode == "F":
-        delta = _bisect(frac, float(p.mean()), -span, span)
-    else:
-        delta = _bisect(recall, cfg.recall, -span, span)
+    deltas = {"F": _bisect(frac, float(p.mean()), -span, span),
+              "R": _bisect(recall, cfg.recall, -span, span)}
+    stats = {m: {"pred_frac": frac(dl), "recall": recall(dl)} for m, dl in deltas.items()}
+    delta = deltas[mode]
 
     bias = torch.tensor(b, dtype=torch.float32, device=device)
     b2 = torch.tensor(b + delta, dtype=torch.float32, device=device)
@@ -254,8 +257,20 @@ def make_layer(cfg: Config, layer: int, device="cpu", mode: str = "R") -> LayerD
         b_up=None if cfg.act == "reglu" else bias,
         b_gate=bias if cfg.act == "reglu" else None,
         p=p, delta=delta,
-        expected_pred_frac=frac(delta), expected_recall=recall(delta),
+        expected_pred_frac=stats[mode]["pred_frac"], expected_recall=stats[mode]["recall"],
+        bias64=b, deltas=deltas, stats=stats,
     )
+
+
+def with_mode(L: LayerData, mode: str) -> LayerData:
+    """The same layer with the predictor bias of the other calibration mode."""
+    kw = dict(L.__dict__)
+    kw["mode"] = mode
+    kw["delta"] = L.deltas[mode]
+    kw["b2"] = torch.tensor(L.bias64 + L.deltas[mode], dtype=torch.float32, device=L.b2.device)
+    kw["expected_pred_frac"] = L.stats[mode]["pred_frac"]
+    kw["expected_recall"] = L.stats[mode]["recall"]
+    return LayerData(**kw)
 
 
 def make_tokens(cfg: Config, n: int, device="cpu", seed_offset: int = 0) -> torch.Tensor:

@@ -1,0 +1,340 @@
+"""GPU parity: every C-ABI call against the fp64 oracle on the same seeded inputs.
+
+Tolerances (written here, derived in the design notes):
+* index lists: bit-exact, except neurons whose oracle logit lies within 1e-3
+  of the threshold, which are excluded and counted;
+* logits: |s_gpu - s| <= 1e-5 * M_n with M_n = sum_j |W2_nj a_j| (+ the
+  propagated first-layer magnitude), a bound on fp32 accumulation error;
+* FFN outputs: relative L2 <= 1e-3 for fp16/bf16 weights, <= 2e-3 for Q4_0;
+* compaction: bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth.configs import Config
+from tests._util import bits_to_bool, device_layer, oracle_layer, raw, rel_l2, to16
+
+pytestmark = pytest.mark.gpu
+
+# small layers spanning every kernel variant (fused and batched paths, ragged
+# unit counts per thread, neuron groups and CTAs)
+SMALL = {
+    c.name: c for c in [
+        synth.get_config("toy"),
+        Config(10, "t-relu-f16-2560", 3, 2560, 4096, "relu", "f16", "f16", 0.02, 1.1, 0.2, 256),
+        Config(11, "t-reglu-bf16", 3, 512, 2048, "reglu", "bf16", "bf16", 0.02, 1.2, 0.12, 128),
+        Config(12, "t-relu-bf16-1024", 2, 1024, 4096, "relu", "bf16", "bf16", 0.02, 1.1, 0.2, 256),
+        Config(13, "t-q4-reglu", 3, 512, 1536, "reglu", "q4_0", "f16", 0.015, 1.1, 0.1, 128),
+        Config(14, "t-q4-relu", 2, 768, 2048, "relu", "q4_0", "f16", 0.015, 1.1, 0.1, 256),
+        Config(15, "t-relu-f16-8192", 2, 8192, 1024, "relu", "f16", "f16", 0.015, 1.0, 0.08, 512),
+    ]
+}
+BATCHES = [1, 2, 4, 8, 32]
+
+
+def ftol(cfg):
+    return 2e-3 if cfg.wdtype == "q4_0" else 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from activation_sparse_pi_b200 import build
+    build.build()
+    import activation_sparse_pi_b200 as pi
+    pi.lib()
+    yield
+    assert pi.pi_device_error() == 0
+
+
+@pytest.fixture(autouse=True)
+def _no_device_error():
+    import activation_sparse_pi_b200 as pi
+    yield
+    assert pi.pi_device_error() == 0, "a kernel flagged a device-side error"
+
+
+_LAYERS = {}
+
+
+def small_layer(name, layer=0):
+    key = (name, layer)
+    if key not in _LAYERS:
+        cfg = SMALL[name]
+        L = synth.make_layer(cfg, layer, "cpu", "R")
+        _LAYERS[key] = (L, oracle_layer(L))
+    return _LAYERS[key]
+
+
+def workspace(descs, B):
+    import activation_sparse_pi_b200 as pi
+    n = pi.pi_workspace_size(descs, B)
+    assert n > 0, pi.pi_last_error()
+    return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+
+def tokens(cfg, B, offset=0):
+    x = synth.make_tokens(cfg, B, seed_offset=offset)
+    return x, x.double().numpy()
+
+
+def run_predict(desc, x16, B, F):
+    import activation_sparse_pi_b200 as pi
+    ws = workspace([desc], B)
+    mask = torch.zeros(B, F // 32, dtype=torch.int32, device="cuda")
+    logits = torch.empty(B, F, dtype=torch.float32, device="cuda")
+    pi.pi_predict(desc.pred, x16, B, mask, logits, ws)
+    torch.cuda.synchronize()
+    return mask.cpu().numpy(), logits.cpu().double().numpy()
+
+
+def logit_bound(OL, x):
+    """Per (token, neuron) magnitude M for the fp32 accumulation bound."""
+    w1 = np.abs(oracle.widen(OL.w1, OL.pdtype))
+    w2 = np.abs(oracle.widen(OL.w2, OL.pdtype))
+    a_mag = np.abs(x) @ w1.T + (np.abs(OL.b1) if OL.b1 is not None else 0)
+    return a_mag @ w2.T + np.abs(OL.b2)
+
+
+def check_index_list(gpu_idx, s_or, thr, I_or):
+    band_any = oracle.band(s_or, thr).any(axis=0)
+    diff = np.setxor1d(gpu_idx, I_or)
+    assert band_any[diff].all(), f"index mismatch outside the 1e-3 band: {diff[~band_any[diff]]}"
+    return diff
+
+
+# ----------------------------------------------------------------- compaction
+@pytest.mark.parametrize("B,F", [(1, 32), (1, 2048), (3, 4096), (8, 16384), (32, 28672),
+                                 (64, 65536), (1, 65536)])
+@pytest.mark.parametrize("density", [0.0, 0.003, 0.3, 1.0])
+def test_compact_bitexact(B, F, density):
+    import activation_sparse_pi_b200 as pi
+    rng = np.random.default_rng(B * 7 + F + int(density * 1000))
+    m = rng.random((B, F)) < density
+    words = np.packbits(m.reshape(B, F // 8, 8)[:, :, ::-1], axis=-1).reshape(B, F // 32, 4)
+    words = words[:, :, ::-1].copy().view(">u4").astype(np.uint32).reshape(B, F // 32)
+    assert np.array_equal(bits_to_bool(words, F), m)
+    mask = torch.from_numpy(words.view(np.int32)).cuda()
+    idx = torch.full((F,), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pi.pi_compact(mask, B, F, idx, cnt)
+    K = int(cnt.item())
+    expect = oracle.union_index(m)
+    assert K == expect.size
+    assert np.array_equal(idx[:K].cpu().numpy(), expect)
+    assert (idx[K:] == -7).all()
+
+
+# ------------------------------------------------------------------ predictor
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("B", BATCHES)
+def test_predict_parity(name, B):
+    L, OL = small_layer(name)
+    cfg = L.cfg
+    Ld, desc = device_layer(L)
+    x, xd = tokens(cfg, B)
+    mask, s_gpu = run_predict(desc, to16(x, cfg.adtype).cuda(), B, cfg.d_ff)
+    _, s_or, m_or = oracle.predict(OL, xd)
+    M = logit_bound(OL, xd)
+    err = np.abs(s_gpu - s_or)
+    assert (err <= 1e-5 * M + 1e-7).all(), float((err / M).max())
+    m_gpu = bits_to_bool(mask, cfg.d_ff)
+    outside = ~oracle.band(s_or, OL.threshold)
+    assert np.array_equal(m_gpu[outside], m_or[outside])
+    assert np.array_equal(m_gpu, s_gpu > OL.threshold)
+
+
+# ---------------------------------------------------------------- sparse FFN
+def run_ffn(desc, x16, B, idx_np, F, d, reps=1):
+    import activation_sparse_pi_b200 as pi
+    ws = workspace([desc], B)
+    idx = torch.zeros(F, dtype=torch.int32, device="cuda")
+    if idx_np.size:
+        idx[: idx_np.size] = torch.from_numpy(idx_np.astype(np.int32)).cuda()
+    cnt = torch.tensor([idx_np.size], dtype=torch.int32, device="cuda")
+    outs = []
+    for _ in range(reps):
+        y = torch.full((B, d), float("nan"), dtype=torch.float32, device="cuda")
+        pi.pi_sparse_ffn(desc, x16, B, idx, cnt, y, ws)
+        torch.cuda.synchronize()
+        outs.append(y.cpu().double().numpy())
+    return outs
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("B", BATCHES)
+@pytest.mark.parametrize("kind", ["predicted", "dense", "few", "shuffled"])
+def test_sparse_ffn_parity(name, B, kind):
+    L, OL = small_layer(name)
+    cfg = L.cfg
+    Ld, desc = device_layer(L)
+    x, xd = tokens(cfg, B, offset=5)
+    F = cfg.d_ff
+    rng = np.random.default_rng(F + B)
+    if kind == "predicted":
+        _, _, m = oracle.predict(OL, xd)
+        I = oracle.union_index(m)
+    elif kind == "dense":
+        I = np.arange(F)
+    elif kind == "few":
+        I = np.sort(rng.choice(F, 5, replace=False))
+    else:
+        _, _, m = oracle.predict(OL, xd)
+        I = rng.permutation(oracle.union_index(m))
+    y1, y2 = run_ffn(desc, to16(x, cfg.adtype).cuda(), B, I, F, cfg.d_model, reps=2)
+    assert np.array_equal(y1, y2), "repeated calls must be bit-identical"
+    expect = oracle.masked_ffn(OL, xd, I)
+    if kind == "dense":
+        np.testing.assert_allclose(oracle.dense_ffn(OL, xd), expect, rtol=1e-12, atol=1e-12)
+    assert rel_l2(y1, expect) <= ftol(cfg), rel_l2(y1, expect)
+
+
+@pytest.mark.parametrize("name", ["toy", "t-reglu-bf16", "t-q4-relu"])
+@pytest.mark.parametrize("B", [1, 8])
+def test_sparse_ffn_empty_index(name, B):
+    L, OL = small_layer(name)
+    cfg = L.cfg
+    Ld, desc = device_layer(L)
+    x, _ = tokens(cfg, B)
+    (y,) = run_ffn(desc, to16(x, cfg.adtype).cuda(), B, np.array([], dtype=np.int64),
+                   cfg.d_ff, cfg.d_model)
+    assert np.all(y == 0.0)
+
+
+def test_bad_index_is_flagged_and_skipped():
+    import activation_sparse_pi_b200 as pi
+    L, OL = small_layer("toy")
+    cfg = L.cfg
+    Ld, desc = device_layer(L)
+    x, xd = tokens(cfg, 1)
+    I = np.array([3, 17, cfg.d_ff + 7, 100, -1, 2047])
+    (y,) = run_ffn(desc, to16(x, cfg.adtype).cuda(), 1, I, cfg.d_ff, cfg.d_model)
+    code = pi.pi_device_error()
+    assert code == 2, code  # out-of-range neuron ids
+    valid = I[(I >= 0) & (I < cfg.d_ff)]
+    assert rel_l2(y, oracle.masked_ffn(OL, xd, valid)) <= 1e-3
+
+
+# ------------------------------------------------------------- whole layer
+def run_layer(desc, x16, B, F, d):
+    import activation_sparse_pi_b200 as pi
+    ws = workspace([desc], B)
+    mask = torch.zeros(B, F // 32, dtype=torch.int32, device="cuda")
+    idx = torch.zeros(F, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = torch.empty(B, d, dtype=torch.float32, device="cuda")
+    pi.pi_predict(desc.pred, x16, B, mask, None, ws)
+    pi.pi_compact(mask, B, F, idx, cnt, ws)
+    pi.pi_sparse_ffn(desc, x16, B, idx, cnt, y, ws)
+    torch.cuda.synchronize()
+    K = int(cnt.item())
+    return idx[:K].cpu().numpy(), y.cpu().double().numpy()
+
+
+def check_layer(L, OL, desc, x, xd, B):
+    cfg = L.cfg
+    gidx, y = run_layer(desc, to16(x, cfg.adtype).cuda(), B, cfg.d_ff, cfg.d_model)
+    _, s_or, m_or = oracle.predict(OL, xd)
+    I_or = oracle.union_index(m_or)
+    diff = check_index_list(gidx, s_or, OL.threshold, I_or)
+    assert np.all(np.diff(gidx) > 0)
+    # with no band disagreement the output is the oracle's own; otherwise the
+    # GPU took another valid decision on band neurons, and its output must be
+    # the masked FFN of that valid list
+    ref_idx = I_or if diff.size == 0 else gidx
+    err = rel_l2(y, oracle.masked_ffn(OL, xd, ref_idx))
+    assert err <= ftol(cfg), err
+    return gidx.size, diff.size
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("B", BATCHES)
+def test_layer_pipeline(name, B):
+    L, OL = small_layer(name)
+    Ld, desc = device_layer(L)
+    x, xd = tokens(L.cfg, B, offset=9)
+    check_layer(L, OL, desc, x, xd, B)
+
+
+# ------------------------------------------------------------------- stack
+def check_stack(layers_or, descs, cfg, x0, B, tol):
+    import activation_sparse_pi_b200 as pi
+    F, nl = cfg.d_ff, len(descs)
+    ws = workspace(descs, B)
+    xr = x0.clone().cuda()
+    idx = torch.zeros(nl, F, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(nl, dtype=torch.int32, device="cuda")
+    pi.pi_ffn_stack(descs, xr, B, idx, cnt, ws)
+    torch.cuda.synchronize()
+    out_or, trace = oracle.ffn_stack(layers_or, x0.double().numpy(), cfg.adtype)
+    gi, gc = idx.cpu().numpy(), cnt.cpu().numpy()
+    for l, (I_or, s_or, _) in enumerate(trace):
+        g = gi[l, : gc[l]]
+        diff = check_index_list(g, s_or, layers_or[l].threshold, I_or)
+        if diff.size:
+            return l  # a band decision differs; later layers see other inputs
+    err = rel_l2(xr.cpu().double().numpy(), out_or)
+    assert err <= tol, err
+    return None
+
+
+@pytest.mark.parametrize("name", [n for n in SMALL if SMALL[n].n_layers > 1])
+@pytest.mark.parametrize("B", [1, 2, 8])
+def test_stack_parity(name, B):
+    cfg = SMALL[name]
+    pairs = [small_layer(name, l) for l in range(cfg.n_layers)]
+    devs = [device_layer(L) for L, _ in pairs]
+    x0 = synth.make_tokens(cfg, B, seed_offset=33)
+    check_stack([OL for _, OL in pairs], [d for _, d in devs], cfg, x0, B, ftol(cfg))
+
+
+def test_stack_deterministic():
+    import activation_sparse_pi_b200 as pi
+    cfg = SMALL["t-relu-f16-2560"]
+    devs = [device_layer(small_layer(cfg.name, l)[0]) for l in range(cfg.n_layers)]
+    descs = [d for _, d in devs]
+    ws = workspace(descs, 1)
+    outs = []
+    for _ in range(3):
+        xr = synth.make_tokens(cfg, 1).cuda()
+        pi.pi_ffn_stack(descs, xr, 1, None, None, ws)
+        outs.append(xr.cpu())
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
+# ------------------------------------------------- full sizes (sampled)
+FULL_LAYER_CASES = [("opt-6.7b", 1), ("opt-6.7b", 4), ("relu-llama2-13b", 1),
+                    ("relu-llama2-13b", 8), ("falcon-40b", 1), ("falcon-40b", 64),
+                    ("llama2-70b-q4", 1), ("llama2-70b-q4", 8), ("llama2-70b-q4", 32)]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,B", FULL_LAYER_CASES)
+def test_full_size_layer(name, B):
+    """One full-size layer of each workload, every output checked."""
+    cfg = synth.get_config(name)
+    L = synth.make_layer(cfg, 1, "cuda", "R")
+    OL = oracle_layer(L)
+    Ld, desc = device_layer(L)
+    x, xd = tokens(cfg, B, offset=77)
+    K, nband = check_layer(L, OL, desc, x, xd, B)
+    assert 0 < K <= cfg.d_ff
+    del L, Ld, desc
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+def test_full_size_opt_stack():
+    """The whole 32-layer OPT-6.7B-shaped stack at batch 1 (the benchmarked
+    launch configuration), one token, against the oracle's own stack."""
+    cfg = synth.get_config("opt-6.7b")
+    layers = [synth.make_layer(cfg, l, "cuda", "R") for l in range(cfg.n_layers)]
+    devs = [device_layer(L) for L in layers]
+    x0 = synth.make_tokens(cfg, 1, seed_offset=101)
+    ors = [oracle_layer(L) for L in layers]
+    first_flip = check_stack(ors, [d for _, d in devs], cfg, x0, 1, 1e-3)
+    assert first_flip is None or first_flip >= 0
+    del layers, devs
+    torch.cuda.empty_cache()
