@@ -64,10 +64,18 @@ int num_sms() {
 constexpr size_t kSmemMax = 227 * 1024;
 constexpr size_t kSmemPred1 = 96 * 1024;
 constexpr size_t kSmemPred2 = 160 * 1024;
-constexpr size_t kSmemFfn = 180 * 1024;
+constexpr size_t kSmemFfn = 220 * 1024;  // shared by the CTAs on one SM
 constexpr size_t kPartCap = 64ull << 20;  // bytes of batched down partials
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// The fused FFN kernel runs ffn_cps(B) CTAs per SM, each with 8 consumer warps
+// and a producer warp whose kFfnProducerLanes lanes issue the bulk copies:
+// measured on B200, one thread issuing 4-8 KB bulk copies cannot keep HBM
+// busy, while several issuing threads per SM can.  Batch 1 fits two CTAs per
+// SM in registers; larger batches keep one.
+constexpr int kFfnProducerLanes = 2;
+int ffn_cps(int B) { return B == 1 ? 2 : 1; }
 
 // ------------------------------------------------------------ workspace
 struct WsLayout {
@@ -91,7 +99,7 @@ WsLayout ws_layout(int d, int F, int r, int B) {
   w.idx = o;   o += al256((size_t)F * 4);
   w.count = o; o += 256;
   w.xl = o;    o += al256((size_t)B * d * 2);
-  const int G = std::max(nsm, down_slices(d, B, nsm));
+  const int G = std::max(ffn_cps(B) * nsm, down_slices(d, B, nsm));
   w.part = o;  o += al256((size_t)G * B * d * 4);
   w.h = o;     o += al256((size_t)F * B * 4);
   w.total = o;
@@ -360,70 +368,106 @@ int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const fl
 }
 
 // ------------------------------------------------------------ gathered FFN
-int cpt_for(int wdt, int d) {
+int ffn_ncw(int wdt, int B) { (void)wdt; (void)B; return 8; }
+int ffn_grid(int B) { return ffn_cps(B) * num_sms(); }
+
+int cpt_for(int wdt, int d, int B) {
   const int units = wdt == PI_Q4_0 ? d / 32 : d / 8;
-  const int need = (units + kConsumers - 1) / kConsumers;
+  const int nct = 32 * ffn_ncw(wdt, B);
+  const int need = (units + nct - 1) / nct;
   for (int c : {1, 2, 4})
     if (c >= need) return c;
   return 0;
 }
 
-int ffn_nstages(const pi_layer* L) {
-  const size_t rb = L->wdtype == PI_Q4_0 ? (size_t)L->d_model / 32 * 18 : (size_t)L->d_model * 2;
-  const size_t stage = rb * (L->act == PI_REGLU ? 3 : 2);
-  const size_t fixed = 1024 + 4096;
-  return (int)std::min<size_t>(32, (kSmemFfn - fixed) / stage);
+size_t ffn_row_bytes(const pi_layer* L) {
+  return L->wdtype == PI_Q4_0 ? (size_t)L->d_model / 32 * 18 : (size_t)L->d_model * 2;
+}
+
+int ffn_list_cap(const pi_layer* L, int B) {
+  return (L->d_ff + ffn_grid(B) - 1) / ffn_grid(B) + 1;
+}
+
+size_t ffn_fixed_smem(const pi_layer* L, int B) {
+  const int ncw = ffn_ncw(L->wdtype, B);
+  const int V = kGroup * (L->act == PI_REGLU ? 2 : 1) * B;
+  return 1024 + (size_t)ffn_list_cap(L, B) * 8 + (size_t)2 * ncw * V * 4 + (size_t)2 * kGroup * B * 4 +
+         128;
+}
+
+int ffn_nstages(const pi_layer* L, int B) {
+  const size_t stage = ffn_row_bytes(L) * (L->act == PI_REGLU ? 3 : 2);
+  const size_t fixed = ffn_fixed_smem(L, B);
+  const size_t budget = kSmemFfn / ffn_cps(B);
+  if (fixed >= budget) return 0;
+  int ns = (int)std::min<size_t>(32, (budget - fixed) / stage);
+  return ns - ns % kFfnProducerLanes;  // each producer lane owns whole stages
 }
 
 bool ffn_fused_ok(const pi_layer* L, int B) {
   if (!(B == 1 || B == 2 || B == 4)) return false;
-  const int c = cpt_for(L->wdtype, L->d_model);
+  const int c = cpt_for(L->wdtype, L->d_model, B);
   if (c == 0) return false;
   if (L->wdtype == PI_Q4_0 ? (B * c > 2) : (B * c > 8)) return false;
-  return ffn_nstages(L) >= kGroup;
+  return ffn_nstages(L, B) >= kGroup;
 }
 
-template <int WDT, int ACT, int B, int CPT>
-cudaError_t launch_ffn(const pi_layer* L, const uint16_t* x, const int32_t* idx,
-                       const int32_t* count, float* part, cudaStream_t st) {
+struct FfnSrc {            // where the fused kernel takes its neuron list from
+  const int32_t* idx;      // explicit list ...
+  const int32_t* count;
+  const uint32_t* mask;    // ... or the predictor's mask bits
+  int mask_rows;
+  int32_t* idx_out;        // mask mode: write the ascending list / count here
+  int32_t* count_out;
+};
+
+template <int WDT, int ACT, int B, int CPT, int NCW>
+cudaError_t launch_ffn(const pi_layer* L, const uint16_t* x, const FfnSrc& src, float* part,
+                       cudaStream_t st) {
   FfnParams p{};
   p.w_act = static_cast<const uint8_t*>(ACT == 1 ? L->w_gate : L->w_up);
   p.w_up = static_cast<const uint8_t*>(L->w_up);
   p.w_dn = static_cast<const uint8_t*>(L->w_down_t);
   p.b_act = ACT == 1 ? L->b_gate : L->b_up;
   p.x = x;
-  p.idx = idx;
-  p.count = count;
+  p.idx = src.idx;
+  p.count = src.count;
+  p.mask = src.mask;
+  p.mask_rows = src.mask_rows;
+  p.idx_out = src.idx_out;
+  p.count_out = src.count_out;
   p.part = part;
   p.d = L->d_model;
   p.F = L->d_ff;
-  p.row_bytes = WDT == 2 ? (uint32_t)(L->d_model / 32 * 18) : (uint32_t)(L->d_model * 2);
-  p.nstages = ffn_nstages(L);
-  const size_t smem = 1024 + 4096 + (size_t)p.nstages * p.row_bytes * (ACT == 1 ? 3 : 2);
-  return launch(k_ffn<WDT, ACT, B, CPT>, dim3(num_sms()), dim3(kThreads), smem, st, p);
+  p.row_bytes = (uint32_t)ffn_row_bytes(L);
+  p.nstages = ffn_nstages(L, B);
+  p.list_cap = ffn_list_cap(L, B);
+  const size_t smem = ffn_fixed_smem(L, B) + (size_t)p.nstages * p.row_bytes * (ACT == 1 ? 3 : 2);
+  return launch(k_ffn<WDT, ACT, B, CPT, NCW, kFfnProducerLanes>, dim3(ffn_grid(B)),
+                dim3(32 * (NCW + 1)), smem, st, p);
 }
 
 template <int WDT, int ACT, int B>
-cudaError_t ffn_cpt(const pi_layer* L, const uint16_t* x, const int32_t* idx, const int32_t* count,
-                    float* part, cudaStream_t st) {
-  const int c = cpt_for(L->wdtype, L->d_model);
+cudaError_t ffn_cpt(const pi_layer* L, const uint16_t* x, const FfnSrc& src, float* part,
+                    cudaStream_t st) {
+  const int c = cpt_for(L->wdtype, L->d_model, B);
   if constexpr (WDT == 2) {
-    if (c == 1) return launch_ffn<WDT, ACT, B, 1>(L, x, idx, count, part, st);
+    if (c == 1) return launch_ffn<WDT, ACT, B, 1, 8>(L, x, src, part, st);
   } else {
-    if (c == 1) return launch_ffn<WDT, ACT, B, 1>(L, x, idx, count, part, st);
-    if (c == 2 && B <= 4) return launch_ffn<WDT, ACT, B, 2>(L, x, idx, count, part, st);
+    if (c == 1) return launch_ffn<WDT, ACT, B, 1, 8>(L, x, src, part, st);
+    if (c == 2) return launch_ffn<WDT, ACT, B, 2, 8>(L, x, src, part, st);
     if constexpr (B <= 2)
-      if (c == 4) return launch_ffn<WDT, ACT, B, 4>(L, x, idx, count, part, st);
+      if (c == 4) return launch_ffn<WDT, ACT, B, 4, 8>(L, x, src, part, st);
   }
   return cudaErrorInvalidValue;
 }
 
 template <int WDT, int ACT>
-cudaError_t ffn_b(const pi_layer* L, int B, const uint16_t* x, const int32_t* idx,
-                  const int32_t* count, float* part, cudaStream_t st) {
-  if (B == 1) return ffn_cpt<WDT, ACT, 1>(L, x, idx, count, part, st);
-  if (B == 2) return ffn_cpt<WDT, ACT, 2>(L, x, idx, count, part, st);
-  if constexpr (WDT != 2) return ffn_cpt<WDT, ACT, 4>(L, x, idx, count, part, st);
+cudaError_t ffn_b(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, float* part,
+                  cudaStream_t st) {
+  if (B == 1) return ffn_cpt<WDT, ACT, 1>(L, x, src, part, st);
+  if (B == 2) return ffn_cpt<WDT, ACT, 2>(L, x, src, part, st);
+  if constexpr (WDT != 2) return ffn_cpt<WDT, ACT, 4>(L, x, src, part, st);
   return cudaErrorInvalidValue;
 }
 
@@ -448,40 +492,53 @@ cudaError_t launch_up_generic(const pi_layer* L, int B, const uint16_t* x, const
   return launch(k_rows<kModeUp, WDT, ACT, 64>, dim3(blocks), dim3(256), 0, st, p);
 }
 
-// mode 0: y = FFN(x); mode 1: out += FFN(x).  ev (optional): two events recorded
-// right before and right after the gathered-FFN kernel.
-int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const int32_t* idx,
-                 const int32_t* count, float* out, int mode, const WsLayout& w, uint8_t* ws,
-                 cudaStream_t st, void* const* ev = nullptr) {
-  if (ev) PI_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(ev[0]), st));
+// Records a caller's timing event on the stream; under stream capture it
+// becomes an external event-record node, so every graph launch records it.
+cudaError_t record_event(void* ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  if (cs == cudaStreamCaptureStatusActive)
+    return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev), st, cudaEventRecordExternal);
+  return cudaEventRecord(static_cast<cudaEvent_t>(ev), st);
+}
+
+// The gathered FFN: mode 0 writes y = FFN(x), mode 1 adds FFN(x) into out.
+// The neuron list is src.idx/src.count, or (fused path only) src.mask.
+// ev (optional): two events recorded right before and after the FFN kernel(s).
+int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, float* out,
+                 int mode, const WsLayout& w, uint8_t* ws, cudaStream_t st,
+                 void* const* ev = nullptr) {
   float* part = reinterpret_cast<float*>(ws + w.part);
   const int d = L->d_model;
   const int n4 = B * d / 4;
   int G;
+  if (ev) PI_CUDA(record_event(ev[0], st));
   if (ffn_fused_ok(L, B)) {
     cudaError_t e = cudaErrorInvalidValue;
     const int act = L->act;
     switch (L->wdtype) {
-      case PI_F16: e = act ? ffn_b<0, 1>(L, B, x, idx, count, part, st) : ffn_b<0, 0>(L, B, x, idx, count, part, st); break;
-      case PI_BF16: e = act ? ffn_b<1, 1>(L, B, x, idx, count, part, st) : ffn_b<1, 0>(L, B, x, idx, count, part, st); break;
-      case PI_Q4_0: e = act ? ffn_b<2, 1>(L, B, x, idx, count, part, st) : ffn_b<2, 0>(L, B, x, idx, count, part, st); break;
+      case PI_F16: e = act ? ffn_b<0, 1>(L, B, x, src, part, st) : ffn_b<0, 0>(L, B, x, src, part, st); break;
+      case PI_BF16: e = act ? ffn_b<1, 1>(L, B, x, src, part, st) : ffn_b<1, 0>(L, B, x, src, part, st); break;
+      case PI_Q4_0: e = act ? ffn_b<2, 1>(L, B, x, src, part, st) : ffn_b<2, 0>(L, B, x, src, part, st); break;
     }
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "fused FFN launch failed: %s", cudaGetErrorString(e));
-    G = num_sms();
+    G = ffn_grid(B);
   } else {
+    if (src.mask) return fail(PI_ERR_UNSUPPORTED, "mask-driven FFN needs the fused kernel");
     float* h = reinterpret_cast<float*>(ws + w.h);
     cudaError_t e = cudaErrorInvalidValue;
     const int act = L->act;
     switch (L->wdtype) {
-      case PI_F16: e = act ? launch_up_generic<0, 1>(L, B, x, idx, count, h, st) : launch_up_generic<0, 0>(L, B, x, idx, count, h, st); break;
-      case PI_BF16: e = act ? launch_up_generic<1, 1>(L, B, x, idx, count, h, st) : launch_up_generic<1, 0>(L, B, x, idx, count, h, st); break;
-      case PI_Q4_0: e = act ? launch_up_generic<2, 1>(L, B, x, idx, count, h, st) : launch_up_generic<2, 0>(L, B, x, idx, count, h, st); break;
+      case PI_F16: e = act ? launch_up_generic<0, 1>(L, B, x, src.idx, src.count, h, st) : launch_up_generic<0, 0>(L, B, x, src.idx, src.count, h, st); break;
+      case PI_BF16: e = act ? launch_up_generic<1, 1>(L, B, x, src.idx, src.count, h, st) : launch_up_generic<1, 0>(L, B, x, src.idx, src.count, h, st); break;
+      case PI_Q4_0: e = act ? launch_up_generic<2, 1>(L, B, x, src.idx, src.count, h, st) : launch_up_generic<2, 0>(L, B, x, src.idx, src.count, h, st); break;
     }
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "batched up launch failed: %s", cudaGetErrorString(e));
     DownParams dp{};
     dp.w_dn = static_cast<const uint8_t*>(L->w_down_t);
-    dp.idx = idx;
-    dp.count = count;
+    dp.idx = src.idx;
+    dp.count = src.count;
     dp.h = h;
     dp.part = part;
     dp.d = d;
@@ -496,7 +553,7 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const int32_t* idx
     }
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "batched down launch failed: %s", cudaGetErrorString(e));
   }
-  if (ev) PI_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(ev[1]), st));
+  if (ev) PI_CUDA(record_event(ev[1], st));
   const dim3 rg((n4 + 31) / 32);
   if (mode == 0) PI_CUDA((launch(k_reduce<0>, rg, dim3(256), 0, st, (const float*)part, G, n4, out)));
   else PI_CUDA((launch(k_reduce<1>, rg, dim3(256), 0, st, (const float*)part, G, n4, out)));
@@ -588,7 +645,8 @@ int32_t pi_sparse_ffn(const pi_layer* layer, const void* x, int32_t batch, const
     return fail(PI_ERR_INVALID_ARG, "x, idx and y must be 16-byte aligned, count 4-byte aligned");
   const WsLayout w = ws_layout(layer->d_model, layer->d_ff, layer->pred.rank, batch);
   if (int32_t s = check_ws(workspace, workspace_bytes, w.total)) return s;
-  return ffn_impl(layer, batch, static_cast<const uint16_t*>(x), idx, count, y, 0, w,
+  FfnSrc src{idx, count, nullptr, 0, nullptr, nullptr};
+  return ffn_impl(layer, batch, static_cast<const uint16_t*>(x), src, y, 0, w,
                   static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
@@ -633,11 +691,18 @@ int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_re
                     ? predict_impl<0>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, st)
                     : predict_impl<1>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, st);
     if (s) return s;
-    PI_CUDA((launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, (const uint32_t*)mask,
-                    (int)batch, L->d_ff, idx, cnt)));
     if (ffn_events && (!ffn_events[2 * l] || !ffn_events[2 * l + 1]))
       return fail(PI_ERR_INVALID_ARG, "ffn_events[%d..%d] must be events", 2 * l, 2 * l + 1);
-    if ((s = ffn_impl(L, batch, xl, idx, cnt, x_resid, 1, w, ws, st,
+    FfnSrc src{idx, cnt, nullptr, 0, nullptr, nullptr};
+    if (ffn_fused_ok(L, batch)) {
+      // compaction fused into the FFN kernel: it reads the mask bits directly
+      src = FfnSrc{nullptr, nullptr, mask, (int)batch, idx_out ? idx : nullptr,
+                   count_out ? cnt : nullptr};
+    } else {
+      PI_CUDA((launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, (const uint32_t*)mask,
+                      (int)batch, L->d_ff, idx, cnt)));
+    }
+    if ((s = ffn_impl(L, batch, xl, src, x_resid, 1, w, ws, st,
                       ffn_events ? ffn_events + 2 * l : nullptr)))
       return s;
   }

@@ -16,6 +16,11 @@ constexpr int kMaxBatch = 64;
 constexpr int kErrTimeout = 1;
 constexpr int kErrBadIndex = 2;
 constexpr uint32_t kWaitLimit = 1u << 22;
+// Suspend-hinted waits: each poll may sleep up to kSuspendNs before returning,
+// so a waiting warp does not spin; kWaitLimitSleep polls bound the wait to
+// about one second.
+constexpr uint32_t kSuspendNs = 2000;
+constexpr uint32_t kWaitLimitSleep = 1u << 19;
 
 // Device error word (read and cleared by pi_device_error()).
 __device__ int g_dev_error;
@@ -55,6 +60,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait that lets the thread sleep between polls.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kWaitLimitSleep; ++it)
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+  set_error(kErrTimeout);
+  return false;
+}
+
 // Bounded wait for the phase with the given parity to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   for (uint32_t it = 0; it < kWaitLimit; ++it)

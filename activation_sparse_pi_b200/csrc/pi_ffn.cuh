@@ -75,14 +75,19 @@ __global__ void __launch_bounds__(kCompactThreads, 1)
 }
 
 // ------------------------------------------------------ gathered FFN, fused
-// Each CTA takes a contiguous, balanced slice [k0, k1) of the K listed
-// neurons.  A stage holds one neuron: its activation row (W_up for ReLU,
-// W_gate for ReGLU), its W_up row (ReGLU only) and its W_down^T row.  The
-// consumers compute h for a group of kGroup neurons (block-wide dot products),
-// then add h * W_down^T[n] into fp32 accumulators that stay in registers for
-// the whole slice.  The CTA's partial y goes to part[cta]; a fixed-order
-// reduction (k_reduce) sums the partials, so there are no atomics and the
-// result is bit-reproducible.
+// Each CTA takes a contiguous, balanced slice [k0, k1) of the K active
+// neurons.  The list comes either from the caller (idx, count) or straight
+// from the predictor's mask bits: every CTA scans the (batch-OR of the) mask
+// words itself, so the index list never round-trips through another kernel;
+// the CTA stages its slice of neuron ids and their biases in shared memory.
+//
+// A stage holds one neuron: its activation row (W_up for ReLU, W_gate for
+// ReGLU), its W_up row (ReGLU only) and its W_down^T row, each one contiguous
+// 1-D bulk copy issued by the producer warp.  The consumer warps compute h for
+// a group of kGroup neurons (block-wide dot products: x stays in registers),
+// then add h * W_down^T[n] into fp32 accumulators held in registers for the
+// whole slice.  The CTA's partial y goes to part[cta]; k_reduce sums the
+// partials in a fixed order, so there are no atomics and y is reproducible.
 constexpr int kGroup = 4;
 
 struct FfnParams {
@@ -91,100 +96,164 @@ struct FfnParams {
   const uint8_t* w_dn;     // W_down^T
   const float* b_act;      // b_up (ReLU) / b_gate (ReGLU), or null
   const uint16_t* x;       // [B x d]
-  const int32_t* idx;
+  const int32_t* idx;      // explicit neuron list (when mask is null)
   const int32_t* count;
+  const uint32_t* mask;    // [mask_rows x F/32] predicted bits, or null
+  int mask_rows;
+  int32_t* idx_out;        // mask mode: the ascending list is written here, or null
+  int32_t* count_out;
   float* part;             // [gridDim.x x B x d]
   int d, F;
   uint32_t row_bytes;
   int nstages;
+  int list_cap;
 };
+
+// Block-wide exclusive scan of one int per thread (all threads of the CTA).
+template <int NT>
+__device__ __forceinline__ int block_excl_scan(int v, int* scratch /* >= 33 ints */, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int t = lane < NT / 32 ? scratch[lane] : 0;
+    int s = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += u;
+    }
+    scratch[lane] = s - t;
+    if (lane == 31) scratch[32] = s;
+  }
+  __syncthreads();
+  total = scratch[32];
+  return scratch[warp] + incl - v;
+}
 
 // WDT: 0 fp16, 1 bf16, 2 Q4_0 (with fp16 activations).  ACT: 0 ReLU, 1 ReGLU.
 // CPT: units per consumer thread (a unit is 8 elements for 16-bit weights, one
-// 32-element block for Q4_0).
-template <int WDT, int ACT, int B, int CPT>
-__global__ void __launch_bounds__(kThreads, 1) k_ffn(FfnParams p) {
+// 32-element block for Q4_0).  NCW: consumer warps.
+// PL: producer lanes.  Lane j issues the copies of items i = j (mod PL), and
+// the stage count is a multiple of PL, so every stage is refilled by one lane
+// only (each lane waits on a stage's phases in order).  Several issuing lanes
+// raise the rate of 1-D bulk copies a CTA can have in flight.
+template <int WDT, int ACT, int B, int CPT, int NCW, int PL>
+__global__ void __launch_bounds__(32 * (NCW + 1), B == 1 ? 2 : 1) k_ffn(FfnParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int NM = ACT == 1 ? 3 : 2;      // matrices per stage
-  constexpr int NUP = ACT == 1 ? 2 : 1;     // dot products per neuron
-  constexpr int V = kGroup * NUP * B;       // values reduced per group
+  constexpr int NT = 32 * (NCW + 1);
+  constexpr int NCT = 32 * NCW;              // consumer threads
+  constexpr int NM = ACT == 1 ? 3 : 2;       // matrices per stage
+  constexpr int NUP = ACT == 1 ? 2 : 1;      // dot products per neuron
+  constexpr int V = kGroup * NUP * B;        // values reduced per group
   constexpr int SH = 5 - log2c<V>();
-  constexpr int XDT = WDT == 1 ? 1 : 0;     // activation dtype
-  constexpr int UE = WDT == 2 ? 32 : 8;     // elements per unit
+  constexpr int XDT = WDT == 1 ? 1 : 0;      // activation dtype
+  constexpr int UE = WDT == 2 ? 32 : 8;      // elements per unit
   const int NS = p.nstages;
 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + NS;
-  float* meta_bias = reinterpret_cast<float*>(empty + NS);     // [NS]
-  int* meta_ok = reinterpret_cast<int*>(meta_bias + NS);       // [NS]
-  float* red = reinterpret_cast<float*>(smem + 1024);          // [2][8][V]
-  float* hs = red + 2 * kConsumerWarps * V;                    // [2][kGroup * B]
-  uint8_t* stages = smem + 1024 + 2 * kConsumerWarps * V * 4 + 2 * kGroup * B * 4;
-  stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(stages) + 127) & ~uintptr_t(127));
+  int* scratch = reinterpret_cast<int*>(smem + 512);              // 64 ints
+  int* ids = reinterpret_cast<int*>(smem + 1024);                  // [list_cap]
+  float* lbias = reinterpret_cast<float*>(ids + p.list_cap);       // [list_cap]
+  float* red = lbias + p.list_cap;                                 // [2][NCW][V]
+  float* hs = red + 2 * NCW * V;                                   // [2][kGroup * B]
+  uint8_t* stages = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(hs + 2 * kGroup * B) + 127) & ~uintptr_t(127));
   const uint32_t rb = p.row_bytes;
   const uint32_t stage_bytes = rb * NM;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], NCW);
     }
     fence_mbar_init();
   }
   __syncthreads();
   pdl_trigger();
-  pdl_wait();  // idx, count and x come from earlier kernels
+  pdl_wait();  // the list (or mask) and x come from earlier kernels
 
-  int K = *p.count;
-  K = K < 0 ? 0 : (K > p.F ? p.F : K);
+  // ---------------------------------------------- this CTA's neuron slice
   const int G = gridDim.x;
-  const int k0 = (int)(((long long)K * blockIdx.x) / G);
-  const int k1 = (int)(((long long)K * (blockIdx.x + 1)) / G);
+  int k0, k1;
+  if (p.mask) {
+    const int W = p.F / 32;
+    const int wpt = (W + NT - 1) / NT;
+    const int w0 = threadIdx.x * wpt;
+    uint32_t words[8];
+    int mine = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      words[k] = 0u;
+      if (k < wpt && w0 + k < W) {
+        uint32_t m = 0u;
+        for (int b = 0; b < p.mask_rows; ++b) m |= p.mask[(size_t)b * W + w0 + k];
+        words[k] = m;
+        mine += __popc(m);
+      }
+    }
+    int K;
+    int pos = block_excl_scan<NT>(mine, scratch, K);
+    k0 = (int)(((long long)K * blockIdx.x) / G);
+    k1 = (int)(((long long)K * (blockIdx.x + 1)) / G);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && p.count_out) *p.count_out = K;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uint32_t m = words[k];
+      while (m) {
+        const int nid = (w0 + k) * 32 + __ffs(m) - 1;
+        m &= m - 1;
+        if (pos >= k0 && pos < k1) {
+          ids[pos - k0] = nid;
+          lbias[pos - k0] = p.b_act ? p.b_act[nid] : 0.f;
+        }
+        if (p.idx_out && pos >= k0 && pos < k1) p.idx_out[pos] = nid;
+        ++pos;
+      }
+    }
+  } else {
+    int K = *p.count;
+    K = K < 0 ? 0 : (K > p.F ? p.F : K);
+    k0 = (int)(((long long)K * blockIdx.x) / G);
+    k1 = (int)(((long long)K * (blockIdx.x + 1)) / G);
+    for (int i = threadIdx.x; i < k1 - k0; i += NT) {
+      const int nid = p.idx[k0 + i];
+      const bool valid = nid >= 0 && nid < p.F;
+      if (!valid) set_error(kErrBadIndex);
+      ids[i] = valid ? nid : -1;
+      lbias[i] = (valid && p.b_act) ? p.b_act[nid] : 0.f;
+    }
+  }
+  __syncthreads();
   const int n = k1 - k0;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {
     // ---------------------------------------------------------- producer
-    const uint64_t pol = policy_evict_first();
-    bool ok = true;
-    for (int base = 0; base < n && ok; base += 32) {
-      int nid = 0, valid = 0;
-      float bias = 0.f;
-      if (base + lane < n) {
-        nid = p.idx[k0 + base + lane];
-        valid = (nid >= 0 && nid < p.F);
-        if (!valid) {
-          set_error(kErrBadIndex);
-          nid = 0;
-        }
-        bias = (p.b_act && valid) ? p.b_act[nid] : 0.f;
+    if (lane < PL) {
+      const uint64_t pol = policy_evict_first();
+      for (int i = lane; i < n; i += PL) {
+        const int s = i % NS;
+        if (i >= NS && !mbar_wait_sleep(&empty[s], ((i / NS) - 1) & 1)) break;
+        const int nid = ids[i] < 0 ? 0 : ids[i];
+        mbar_arrive_expect_tx(&full[s], stage_bytes);
+        uint8_t* st = stages + (size_t)s * stage_bytes;
+        const size_t off = (size_t)nid * rb;
+        bulk_g2s_hint(st, p.w_act + off, rb, &full[s], pol);
+        if constexpr (ACT == 1) bulk_g2s_hint(st + rb, p.w_up + off, rb, &full[s], pol);
+        bulk_g2s_hint(st + (NM - 1) * rb, p.w_dn + off, rb, &full[s], pol);
       }
-      const int cnt = min(32, n - base);
-      for (int j = 0; j < cnt; ++j) {
-        const int nj = __shfl_sync(0xffffffffu, nid, j);
-        const int vj = __shfl_sync(0xffffffffu, valid, j);
-        const float bj = __shfl_sync(0xffffffffu, bias, j);
-        if (lane == 0 && ok) {
-          const int i = base + j;
-          const int s = i % NS;
-          if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) {
-            ok = false;
-          } else {
-            meta_bias[s] = bj;
-            meta_ok[s] = vj;
-            mbar_arrive_expect_tx(&full[s], stage_bytes);
-            uint8_t* st = stages + (size_t)s * stage_bytes;
-            const size_t off = (size_t)nj * rb;
-            bulk_g2s_hint(st, p.w_act + off, rb, &full[s], pol);
-            if constexpr (ACT == 1) bulk_g2s_hint(st + rb, p.w_up + off, rb, &full[s], pol);
-            bulk_g2s_hint(st + (NM - 1) * rb, p.w_dn + off, rb, &full[s], pol);
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-      }
+      // drain this lane's last copies before the CTA can exit
+      for (int i = lane; i < n; i += PL)
+        if (i >= n - NS) mbar_wait_sleep(&full[i % NS], (i / NS) & 1);
     }
-    if (lane == 0)
-      for (int i = max(0, n - NS); i < n; ++i) mbar_wait(&full[i % NS], (i / NS) & 1);
     return;
   }
 
@@ -193,14 +262,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn(FfnParams p) {
   const int cw = warp - 1;
   const int nunits = p.d / UE;
 
-  // activations of this thread's units, per token
   constexpr int XW = WDT == 2 ? 32 : 4;  // Q4: 32 fp32 values; 16-bit: 4 packed words
   uint32_t xr[B][CPT][XW];
 #pragma unroll
   for (int b = 0; b < B; ++b)
 #pragma unroll
     for (int c = 0; c < CPT; ++c) {
-      const int u = ct + kConsumers * c;
+      const int u = ct + NCT * c;
       if constexpr (WDT == 2) {
 #pragma unroll
         for (int e = 0; e < 32; ++e)
@@ -222,6 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn(FfnParams p) {
 #pragma unroll
       for (int e = 0; e < UE; ++e) acc[b][c][e] = 0.f;
 
+  // Every consumer takes part in every group's barriers, so a timed-out wait
+  // only stops this thread's arithmetic, never its barrier arrivals.
   bool ok = true;
   int grp = 0;
   for (int g = 0; g < n; g += kGroup, ++grp) {
@@ -230,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn(FfnParams p) {
 #pragma unroll
     for (int q = 0; q < kGroup; ++q) {
       const int i = g + q;
-      if (q < ng && ok && !mbar_wait(&full[i % NS], (i / NS) & 1)) ok = false;
+      if (q < ng && ok && !mbar_wait_sleep(&full[i % NS], (i / NS) & 1)) ok = false;
     }
     // partial dot products of this thread's units
     float v[V];
@@ -246,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn(FfnParams p) {
             const uint8_t* row = st + m * rb;
 #pragma unroll
             for (int c = 0; c < CPT; ++c) {
-              const int u = ct + kConsumers * c;
+              const int u = ct + NCT * c;
               if (u < nunits) {
                 if constexpr (WDT == 2) {
                   const uint8_t* blk = row + (size_t)u * 18;
@@ -287,27 +357,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn(FfnParams p) {
     }
     // block reduction: warp transposed reduce, then across warps
     const float tot = warp_reduce_transposed<V>(v);
-    if ((lane & ((1 << SH) - 1)) == 0) red[(buf * kConsumerWarps + cw) * V + (lane >> SH)] = tot;
-    named_bar_sync(1, kConsumers);
+    if ((lane & ((1 << SH) - 1)) == 0) red[(buf * NCW + cw) * V + (lane >> SH)] = tot;
+    named_bar_sync(1, NCT);
     if (ct < kGroup * B) {
       const int q = ct / B, b = ct % B;
       float h = 0.f;
       if (q < ng && ok) {
         float sa = 0.f, su = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          sa += red[(buf * kConsumerWarps + w) * V + (q * NUP + 0) * B + b];
-          if constexpr (ACT == 1) su += red[(buf * kConsumerWarps + w) * V + (q * NUP + 1) * B + b];
+        for (int w = 0; w < NCW; ++w) {
+          sa += red[(buf * NCW + w) * V + (q * NUP + 0) * B + b];
+          if constexpr (ACT == 1) su += red[(buf * NCW + w) * V + (q * NUP + 1) * B + b];
         }
-        const int s = (g + q) % NS;
-        const float pre = sa + meta_bias[s];
-        h = fmaxf(pre, 0.f);
+        const int i = g + q;
+        h = fmaxf(sa + lbias[i], 0.f);
         if constexpr (ACT == 1) h *= su;
-        if (!meta_ok[s]) h = 0.f;
+        if (ids[i] < 0) h = 0.f;
       }
       hs[buf * kGroup * B + ct] = h;
     }
-    named_bar_sync(1, kConsumers);
+    named_bar_sync(1, NCT);
     // down projection: acc += h * W_down^T[n]
     if (ok) {
 #pragma unroll
@@ -319,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn(FfnParams p) {
           for (int b = 0; b < B; ++b) hq[b] = hs[buf * kGroup * B + q * B + b];
 #pragma unroll
           for (int c = 0; c < CPT; ++c) {
-            const int u = ct + kConsumers * c;
+            const int u = ct + NCT * c;
             if (u < nunits) {
               if constexpr (WDT == 2) {
                 const uint8_t* blk = row + (size_t)u * 18;
@@ -367,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn(FfnParams p) {
   for (int b = 0; b < B; ++b)
 #pragma unroll
     for (int c = 0; c < CPT; ++c) {
-      const int u = ct + kConsumers * c;
+      const int u = ct + NCT * c;
       if (u < nunits) {
         float4* dst = reinterpret_cast<float4*>(p.part + ((size_t)blockIdx.x * B + b) * p.d +
                                                 (size_t)u * UE);

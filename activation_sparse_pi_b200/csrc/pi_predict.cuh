@@ -110,13 +110,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_pred1(Pred1Params p) {
     if (lane == 0) {
       for (int i = 0; i < n; ++i) {
         const int s = i % NS;
-        if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) break;
+        if (i >= NS && !mbar_wait_sleep(&empty[s], ((i / NS) - 1) & 1)) break;
         mbar_arrive_expect_tx(&full[s], row_bytes);
         bulk_g2s(stages + (size_t)s * row_bytes, p.w1 + (size_t)(j0 + i) * row_bytes, row_bytes,
                  &full[s]);
       }
       // drain: no copy may still be in flight when the CTA exits
-      for (int i = max(0, n - NS); i < n; ++i) mbar_wait(&full[i % NS], (i / NS) & 1);
+      for (int i = max(0, n - NS); i < n; ++i) mbar_wait_sleep(&full[i % NS], (i / NS) & 1);
     }
     return;
   }
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_pred1(Pred1Params p) {
 #pragma unroll
     for (int q = 0; q < kRowGroup; ++q) {
       const int i = g + q;
-      if (q < ng && ok && !mbar_wait(&full[i % NS], (i / NS) & 1)) ok = false;
+      if (q < ng && ok && !mbar_wait_sleep(&full[i % NS], (i / NS) & 1)) ok = false;
     }
     float v[V];
 #pragma unroll
@@ -253,12 +253,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_pred2(Pred2Params p) {
       const uint8_t* base = p.w2 + (size_t)u0 * 32 * row_bytes;
       for (int i = 0; i < nst; ++i) {
         const int s = i % NS;
-        if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) break;
+        if (i >= NS && !mbar_wait_sleep(&empty[s], ((i / NS) - 1) & 1)) break;
         mbar_arrive_expect_tx(&full[s], stage_bytes);
         bulk_g2s(stages + (size_t)s * stage_bytes, base + (size_t)i * stage_bytes, stage_bytes,
                  &full[s]);
       }
-      for (int i = max(0, nst - NS); i < nst; ++i) mbar_wait(&full[i % NS], (i / NS) & 1);
+      for (int i = max(0, nst - NS); i < nst; ++i) mbar_wait_sleep(&full[i % NS], (i / NS) & 1);
     }
     return;
   }
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_pred2(Pred2Params p) {
   for (int ui = 0; ui < nu; ++ui) {
     const int i = ui * 4 + (cw >> 1);  // stage holding rows 4cw..4cw+3
     const int s = i % NS;
-    if (ok && !mbar_wait(&full[s], (i / NS) & 1)) ok = false;
+    if (ok && !mbar_wait_sleep(&full[s], (i / NS) & 1)) ok = false;
     float v[V];
 #pragma unroll
     for (int q = 0; q < V; ++q) v[q] = 0.f;

@@ -338,3 +338,33 @@ def test_full_size_opt_stack():
     assert first_flip is None or first_flip >= 0
     del layers, devs
     torch.cuda.empty_cache()
+
+
+def test_stack_timed_events():
+    """The timed stack gives the untimed stack's result, and its events time
+    every layer's gathered FFN, eagerly and inside a CUDA graph."""
+    import activation_sparse_pi_b200 as pi
+    cfg = SMALL["t-relu-f16-2560"]
+    devs = [device_layer(small_layer(cfg.name, l)[0]) for l in range(cfg.n_layers)]
+    descs = pi.layer_array([d for _, d in devs])
+    ws = workspace(descs, 1)
+    x0 = synth.make_tokens(cfg, 1).cuda()
+    a = x0.clone()
+    pi.pi_ffn_stack(descs, a, 1, None, None, ws)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cfg.n_layers)]
+    for e in evs:
+        e.record()
+    b = x0.clone()
+    pi.pi_ffn_stack_timed(descs, b, 1, None, None, ws, evs)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert all(evs[2 * l].elapsed_time(evs[2 * l + 1]) > 0 for l in range(cfg.n_layers))
+    c = x0.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        pi.pi_ffn_stack_timed(descs, c, 1, None, None, ws, evs)
+    c.copy_(x0)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(a, c)
+    assert all(evs[2 * l].elapsed_time(evs[2 * l + 1]) > 0 for l in range(cfg.n_layers))
