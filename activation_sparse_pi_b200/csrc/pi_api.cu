@@ -69,13 +69,11 @@ constexpr size_t kPartCap = 64ull << 20;  // bytes of batched down partials
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// The fused FFN kernel runs ffn_cps(B) CTAs per SM, each with 8 consumer warps
-// and a producer warp whose kFfnProducerLanes lanes issue the bulk copies:
-// measured on B200, one thread issuing 4-8 KB bulk copies cannot keep HBM
-// busy, while several issuing threads per SM can.  Batch 1 fits two CTAs per
-// SM in registers; larger batches keep one.
-constexpr int kFfnProducerLanes = 2;
+// The fused FFN kernel runs ffn_cps(B) CTAs of 256 threads per SM: two at
+// batch 1 (registers allow it, and two independent block-reduction domains
+// per SM keep more copies in flight), one for larger batches.
 int ffn_cps(int B) { return B == 1 ? 2 : 1; }
+int ffn_grid(int B);
 
 // ------------------------------------------------------------ workspace
 struct WsLayout {
@@ -368,48 +366,59 @@ int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const fl
 }
 
 // ------------------------------------------------------------ gathered FFN
-int ffn_ncw(int wdt, int B) { (void)wdt; (void)B; return 8; }
 int ffn_grid(int B) { return ffn_cps(B) * num_sms(); }
-
-int cpt_for(int wdt, int d, int B) {
-  const int units = wdt == PI_Q4_0 ? d / 32 : d / 8;
-  const int nct = 32 * ffn_ncw(wdt, B);
-  const int need = (units + nct - 1) / nct;
-  for (int c : {1, 2, 4})
-    if (c >= need) return c;
-  return 0;
-}
 
 size_t ffn_row_bytes(const pi_layer* L) {
   return L->wdtype == PI_Q4_0 ? (size_t)L->d_model / 32 * 18 : (size_t)L->d_model * 2;
 }
 
+int ffn_nm(const pi_layer* L) { return L->act == PI_REGLU ? 3 : 2; }
+
 int ffn_list_cap(const pi_layer* L, int B) {
   return (L->d_ff + ffn_grid(B) - 1) / ffn_grid(B) + 1;
 }
 
-size_t ffn_fixed_smem(const pi_layer* L, int B) {
-  const int ncw = ffn_ncw(L->wdtype, B);
-  const int V = kGroup * (L->act == PI_REGLU ? 2 : 1) * B;
-  return 1024 + (size_t)ffn_list_cap(L, B) * 8 + (size_t)2 * ncw * V * 4 + (size_t)2 * kGroup * B * 4 +
-         128;
+// 16-bit weights (k_ffn_ldg): down-phase column chunks per thread
+int ldg_cpt(int d) {
+  const int need = (d / 8 + kLdgThreads - 1) / kLdgThreads;
+  for (int c : {1, 2, 4})
+    if (c >= need) return c;
+  return 0;
 }
 
-int ffn_nstages(const pi_layer* L, int B) {
-  const size_t stage = ffn_row_bytes(L) * (L->act == PI_REGLU ? 3 : 2);
-  const size_t fixed = ffn_fixed_smem(L, B);
+size_t ldg_smem(const pi_layer* L, int B) {
+  return 256 + (size_t)ffn_list_cap(L, B) * (8 + 4 * B) + 16 + (size_t)B * L->d_model * 4;
+}
+
+// Q4_0 weights (k_ffn_tma): 8 consumer warps, kTmaLanes producer lanes
+constexpr int kTmaNcw = 8;
+constexpr int kTmaLanes = 2;
+
+size_t tma_fixed_smem(const pi_layer* L, int B) {
+  const int V = kGroup * (L->act == PI_REGLU ? 2 : 1) * B;
+  return 1024 + (size_t)ffn_list_cap(L, B) * 8 + (size_t)2 * kTmaNcw * V * 4 +
+         (size_t)2 * kGroup * B * 4 + 128;
+}
+
+int tma_nstages(const pi_layer* L, int B) {
+  const size_t stage = ffn_row_bytes(L) * ffn_nm(L);
+  const size_t fixed = tma_fixed_smem(L, B);
   const size_t budget = kSmemFfn / ffn_cps(B);
   if (fixed >= budget) return 0;
   int ns = (int)std::min<size_t>(32, (budget - fixed) / stage);
-  return ns - ns % kFfnProducerLanes;  // each producer lane owns whole stages
+  return ns - ns % kTmaLanes;  // each producer lane owns whole stages
 }
 
 bool ffn_fused_ok(const pi_layer* L, int B) {
   if (!(B == 1 || B == 2 || B == 4)) return false;
-  const int c = cpt_for(L->wdtype, L->d_model, B);
-  if (c == 0) return false;
-  if (L->wdtype == PI_Q4_0 ? (B * c > 2) : (B * c > 8)) return false;
-  return ffn_nstages(L, B) >= kGroup;
+  if (L->wdtype == PI_Q4_0) {
+    // one 32-element block per consumer thread
+    if (L->d_model / 32 > 32 * kTmaNcw || B > 2) return false;
+    return tma_nstages(L, B) >= kGroup;
+  }
+  const int c = ldg_cpt(L->d_model);
+  if (c == 0 || B * c > 8) return false;
+  return ldg_smem(L, B) <= kSmemFfn / ffn_cps(B);
 }
 
 struct FfnSrc {            // where the fused kernel takes its neuron list from
@@ -421,14 +430,13 @@ struct FfnSrc {            // where the fused kernel takes its neuron list from
   int32_t* count_out;
 };
 
-template <int WDT, int ACT, int B, int CPT, int NCW>
-cudaError_t launch_ffn(const pi_layer* L, const uint16_t* x, const FfnSrc& src, float* part,
-                       cudaStream_t st) {
+FfnParams ffn_params(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, float* part) {
   FfnParams p{};
-  p.w_act = static_cast<const uint8_t*>(ACT == 1 ? L->w_gate : L->w_up);
+  const bool reglu = L->act == PI_REGLU;
+  p.w_act = static_cast<const uint8_t*>(reglu ? L->w_gate : L->w_up);
   p.w_up = static_cast<const uint8_t*>(L->w_up);
   p.w_dn = static_cast<const uint8_t*>(L->w_down_t);
-  p.b_act = ACT == 1 ? L->b_gate : L->b_up;
+  p.b_act = reglu ? L->b_gate : L->b_up;
   p.x = x;
   p.idx = src.idx;
   p.count = src.count;
@@ -440,34 +448,53 @@ cudaError_t launch_ffn(const pi_layer* L, const uint16_t* x, const FfnSrc& src, 
   p.d = L->d_model;
   p.F = L->d_ff;
   p.row_bytes = (uint32_t)ffn_row_bytes(L);
-  p.nstages = ffn_nstages(L, B);
   p.list_cap = ffn_list_cap(L, B);
-  const size_t smem = ffn_fixed_smem(L, B) + (size_t)p.nstages * p.row_bytes * (ACT == 1 ? 3 : 2);
-  return launch(k_ffn<WDT, ACT, B, CPT, NCW, kFfnProducerLanes>, dim3(ffn_grid(B)),
-                dim3(32 * (NCW + 1)), smem, st, p);
+  return p;
+}
+
+template <int WDT, int ACT, int B, int CPT>
+cudaError_t launch_ffn_ldg(const pi_layer* L, const uint16_t* x, const FfnSrc& src, float* part,
+                           cudaStream_t st) {
+  const FfnParams p = ffn_params(L, B, x, src, part);
+  constexpr int CPS = B == 1 ? 2 : 1;
+  return launch(k_ffn_ldg<WDT, ACT, B, CPT, CPS>, dim3(ffn_grid(B)), dim3(kLdgThreads),
+                ldg_smem(L, B), st, p);
 }
 
 template <int WDT, int ACT, int B>
-cudaError_t ffn_cpt(const pi_layer* L, const uint16_t* x, const FfnSrc& src, float* part,
-                    cudaStream_t st) {
-  const int c = cpt_for(L->wdtype, L->d_model, B);
-  if constexpr (WDT == 2) {
-    if (c == 1) return launch_ffn<WDT, ACT, B, 1, 8>(L, x, src, part, st);
-  } else {
-    if (c == 1) return launch_ffn<WDT, ACT, B, 1, 8>(L, x, src, part, st);
-    if (c == 2) return launch_ffn<WDT, ACT, B, 2, 8>(L, x, src, part, st);
-    if constexpr (B <= 2)
-      if (c == 4) return launch_ffn<WDT, ACT, B, 4, 8>(L, x, src, part, st);
+cudaError_t ffn_ldg_cpt(const pi_layer* L, const uint16_t* x, const FfnSrc& src, float* part,
+                        cudaStream_t st) {
+  switch (ldg_cpt(L->d_model)) {
+    case 1: return launch_ffn_ldg<WDT, ACT, B, 1>(L, x, src, part, st);
+    case 2: return launch_ffn_ldg<WDT, ACT, B, 2>(L, x, src, part, st);
+    case 4: if constexpr (B <= 2) return launch_ffn_ldg<WDT, ACT, B, 4>(L, x, src, part, st); break;
   }
   return cudaErrorInvalidValue;
 }
 
 template <int WDT, int ACT>
-cudaError_t ffn_b(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, float* part,
-                  cudaStream_t st) {
-  if (B == 1) return ffn_cpt<WDT, ACT, 1>(L, x, src, part, st);
-  if (B == 2) return ffn_cpt<WDT, ACT, 2>(L, x, src, part, st);
-  if constexpr (WDT != 2) return ffn_cpt<WDT, ACT, 4>(L, x, src, part, st);
+cudaError_t ffn_ldg(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, float* part,
+                    cudaStream_t st) {
+  if (B == 1) return ffn_ldg_cpt<WDT, ACT, 1>(L, x, src, part, st);
+  if (B == 2) return ffn_ldg_cpt<WDT, ACT, 2>(L, x, src, part, st);
+  return ffn_ldg_cpt<WDT, ACT, 4>(L, x, src, part, st);
+}
+
+template <int ACT, int B>
+cudaError_t launch_ffn_tma(const pi_layer* L, const uint16_t* x, const FfnSrc& src, float* part,
+                           cudaStream_t st) {
+  FfnParams p = ffn_params(L, B, x, src, part);
+  p.nstages = tma_nstages(L, B);
+  const size_t smem = tma_fixed_smem(L, B) + (size_t)p.nstages * p.row_bytes * ffn_nm(L);
+  return launch(k_ffn_tma<2, ACT, B, 1, kTmaNcw, kTmaLanes>, dim3(ffn_grid(B)),
+                dim3(32 * (kTmaNcw + 1)), smem, st, p);
+}
+
+template <int ACT>
+cudaError_t ffn_tma(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, float* part,
+                    cudaStream_t st) {
+  if (B == 1) return launch_ffn_tma<ACT, 1>(L, x, src, part, st);
+  if (B == 2) return launch_ffn_tma<ACT, 2>(L, x, src, part, st);
   return cudaErrorInvalidValue;
 }
 
@@ -518,9 +545,9 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     cudaError_t e = cudaErrorInvalidValue;
     const int act = L->act;
     switch (L->wdtype) {
-      case PI_F16: e = act ? ffn_b<0, 1>(L, B, x, src, part, st) : ffn_b<0, 0>(L, B, x, src, part, st); break;
-      case PI_BF16: e = act ? ffn_b<1, 1>(L, B, x, src, part, st) : ffn_b<1, 0>(L, B, x, src, part, st); break;
-      case PI_Q4_0: e = act ? ffn_b<2, 1>(L, B, x, src, part, st) : ffn_b<2, 0>(L, B, x, src, part, st); break;
+      case PI_F16: e = act ? ffn_ldg<0, 1>(L, B, x, src, part, st) : ffn_ldg<0, 0>(L, B, x, src, part, st); break;
+      case PI_BF16: e = act ? ffn_ldg<1, 1>(L, B, x, src, part, st) : ffn_ldg<1, 0>(L, B, x, src, part, st); break;
+      case PI_Q4_0: e = act ? ffn_tma<1>(L, B, x, src, part, st) : ffn_tma<0>(L, B, x, src, part, st); break;
     }
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "fused FFN launch failed: %s", cudaGetErrorString(e));
     G = ffn_grid(B);

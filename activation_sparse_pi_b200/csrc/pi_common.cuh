@@ -138,23 +138,30 @@ __device__ __forceinline__ float2 unpack2(uint32_t u) {
   }
 }
 
-// acc0 += w.lo * x.lo, acc1 += w.hi * x.hi with both operands 16-bit; the
-// products are exact and each accumulation is one fp32 rounding.
+// Only standard fp32 FMAs are used for 16-bit operands (each widened exactly
+// to fp32, so products are exact): an earlier form of these kernels with the
+// mixed-precision fma.f32.bf16 instruction faulted with "illegal instruction"
+// in one kernel instantiation on B200.
+// Sum of the 8 products of a 16-byte chunk of 16-bit weights with 8 fp32
+// activations (two accumulation chains).
 template <int DT>
-__device__ __forceinline__ void dot2(uint32_t w, uint32_t x, float& acc0, float& acc1) {
-  if constexpr (DT == 0) {
-    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
-        "mov.b32 {wl, wh}, %2;\n\tmov.b32 {xl, xh}, %3;\n\t"
-        "fma.rn.f32.f16 %0, wl, xl, %0;\n\tfma.rn.f32.f16 %1, wh, xh, %1;\n\t}"
-        : "+f"(acc0), "+f"(acc1)
-        : "r"(w), "r"(x));
-  } else {
-    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
-        "mov.b32 {wl, wh}, %2;\n\tmov.b32 {xl, xh}, %3;\n\t"
-        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\tfma.rn.f32.bf16 %1, wh, xh, %1;\n\t}"
-        : "+f"(acc0), "+f"(acc1)
-        : "r"(w), "r"(x));
-  }
+__device__ __forceinline__ float dot8(const uint4& w, const float* x) {
+  const float2 f0 = unpack2<DT>(w.x), f1 = unpack2<DT>(w.y);
+  const float2 f2 = unpack2<DT>(w.z), f3 = unpack2<DT>(w.w);
+  float a0 = f0.x * x[0], a1 = f0.y * x[1];
+  a0 = fmaf(f1.x, x[2], a0); a1 = fmaf(f1.y, x[3], a1);
+  a0 = fmaf(f2.x, x[4], a0); a1 = fmaf(f2.y, x[5], a1);
+  a0 = fmaf(f3.x, x[6], a0); a1 = fmaf(f3.y, x[7], a1);
+  return a0 + a1;
+}
+
+// Widen a 16-byte chunk of 16-bit activations to 8 fp32 values.
+template <int DT>
+__device__ __forceinline__ void widen8(const uint4& v, float* x) {
+  const float2 f0 = unpack2<DT>(v.x), f1 = unpack2<DT>(v.y);
+  const float2 f2 = unpack2<DT>(v.z), f3 = unpack2<DT>(v.w);
+  x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
+  x[4] = f2.x; x[5] = f2.y; x[6] = f3.x; x[7] = f3.y;
 }
 
 // Round an fp32 value to the 16-bit activation type (nearest even), as bits.

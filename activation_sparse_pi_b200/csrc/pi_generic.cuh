@@ -143,12 +143,9 @@ __global__ void __launch_bounds__(256) k_rows(RowsParams p) {
                 acc[m][b] = s;
               } else {
                 const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x16 + (size_t)b * p.len + c * 8));
-                float a0 = 0.f, a1 = 0.f;
-                dot2<XDT>(w.x, xv.x, a0, a1);
-                dot2<XDT>(w.y, xv.y, a0, a1);
-                dot2<XDT>(w.z, xv.z, a0, a1);
-                dot2<XDT>(w.w, xv.w, a0, a1);
-                acc[m][b] += a0 + a1;
+                float xf[8];
+                widen8<XDT>(xv, xf);
+                acc[m][b] += dot8<WDT == 2 ? 0 : WDT>(w, xf);
               }
             }
           }

@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_pred1(Pred1Params p) {
   named_bar_sync(1, kConsumers);
 
   const int nchunks = p.d / 8;
-  uint32_t xr[B][CPT][4];
+  float xr[B][CPT][8];  // this thread's activations, widened once to fp32
 #pragma unroll
   for (int b = 0; b < B; ++b)
 #pragma unroll
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_pred1(Pred1Params p) {
       const int u = ct + kConsumers * c;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (u < nchunks) v = *reinterpret_cast<const uint4*>(xs + (size_t)b * p.d + u * 8);
-      xr[b][c][0] = v.x; xr[b][c][1] = v.y; xr[b][c][2] = v.z; xr[b][c][3] = v.w;
+      widen8<DT>(v, xr[b][c]);
     }
 
   bool ok = true;
@@ -170,14 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_pred1(Pred1Params p) {
             if (u < nchunks) {
               const uint4 w = *reinterpret_cast<const uint4*>(row + (size_t)u * 16);
 #pragma unroll
-              for (int b = 0; b < B; ++b) {
-                float a0 = 0.f, a1 = 0.f;
-                dot2<DT>(w.x, xr[b][c][0], a0, a1);
-                dot2<DT>(w.y, xr[b][c][1], a0, a1);
-                dot2<DT>(w.z, xr[b][c][2], a0, a1);
-                dot2<DT>(w.w, xr[b][c][3], a0, a1);
-                v[q * B + b] += a0 + a1;
-              }
+              for (int b = 0; b < B; ++b) v[q * B + b] += dot8<DT>(w, xr[b][c]);
             }
           }
         }
