@@ -72,7 +72,10 @@ size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 // The fused FFN kernel runs ffn_cps(B) CTAs of 256 threads per SM: two at
 // batch 1 (registers allow it, and two independent block-reduction domains
 // per SM keep more copies in flight), one for larger batches.
-int ffn_cps(int B) { return B == 1 ? 2 : 1; }
+#ifndef PI_LDG_CPS
+#define PI_LDG_CPS 2
+#endif
+int ffn_cps(int B) { return B == 1 ? PI_LDG_CPS : 1; }
 int ffn_grid(int B);
 
 // ------------------------------------------------------------ workspace
@@ -118,8 +121,13 @@ cudaError_t launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s
     const auto key = std::make_pair(dev, reinterpret_cast<const void*>(kern));
     std::lock_guard<std::mutex> lock(mu);
     if (!done.count(key)) {
+      // the carve-out is shared with the kernel's static shared memory
+      cudaFuncAttributes fa{};
+      e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kern));
+      if (e != cudaSuccess) return e;
       e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax);
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(kSmemMax - fa.sharedSizeBytes));
       if (e != cudaSuccess) return e;
       done.insert(key);
     }
@@ -456,7 +464,7 @@ template <int WDT, int ACT, int B, int CPT>
 cudaError_t launch_ffn_ldg(const pi_layer* L, const uint16_t* x, const FfnSrc& src, float* part,
                            cudaStream_t st) {
   const FfnParams p = ffn_params(L, B, x, src, part);
-  constexpr int CPS = B == 1 ? 2 : 1;
+  constexpr int CPS = B == 1 ? PI_LDG_CPS : 1;
   return launch(k_ffn_ldg<WDT, ACT, B, CPT, CPS>, dim3(ffn_grid(B)), dim3(kLdgThreads),
                 ldg_smem(L, B), st, p);
 }
@@ -581,9 +589,10 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "batched down launch failed: %s", cudaGetErrorString(e));
   }
   if (ev) PI_CUDA(record_event(ev[1], st));
-  const dim3 rg((n4 + 31) / 32);
-  if (mode == 0) PI_CUDA((launch(k_reduce<0>, rg, dim3(256), 0, st, (const float*)part, G, n4, out)));
-  else PI_CUDA((launch(k_reduce<1>, rg, dim3(256), 0, st, (const float*)part, G, n4, out)));
+  const dim3 rg((n4 + kRedCols - 1) / kRedCols);
+  const dim3 rt(kRedCols * kRedSlices);
+  if (mode == 0) PI_CUDA((launch(k_reduce<0>, rg, rt, 0, st, (const float*)part, G, n4, out)));
+  else PI_CUDA((launch(k_reduce<1>, rg, rt, 0, st, (const float*)part, G, n4, out)));
   return PI_OK;
 }
 

@@ -112,6 +112,12 @@ __device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32
       : "memory");
 }
 
+// Hint the L2 to fetch [src, src + bytes) (16-byte aligned, bytes % 16 == 0);
+// no completion is tracked.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------- programmatic dependent launch
 // Wait until the preceding kernel in the stream has completed and its memory
 // is visible (no-op when the kernel was not launched as a dependent).

@@ -132,7 +132,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch /* >= 33 ints
 // This CTA's slice [k0, k1) of the neuron list, staged in ids / lbias (ids
 // of invalid explicit entries are -1).  All NT threads call it; it ends with a
 // CTA barrier.
-template <int NT>
+template <int NT, bool BIAS = true>
 __device__ void build_slice(const FfnParams& p, int* scratch, int* ids, float* lbias, int& k0,
                             int& k1) {
   const int G = gridDim.x;
@@ -165,7 +165,7 @@ __device__ void build_slice(const FfnParams& p, int* scratch, int* ids, float* l
         m &= m - 1;
         if (pos >= k0 && pos < k1) {
           ids[pos - k0] = nid;
-          lbias[pos - k0] = p.b_act ? p.b_act[nid] : 0.f;
+          if (BIAS) lbias[pos - k0] = p.b_act ? p.b_act[nid] : 0.f;
           if (p.idx_out) p.idx_out[pos] = nid;
         }
         ++pos;
@@ -181,7 +181,7 @@ __device__ void build_slice(const FfnParams& p, int* scratch, int* ids, float* l
       const bool valid = nid >= 0 && nid < p.F;
       if (!valid) set_error(kErrBadIndex);
       ids[i] = valid ? nid : -1;
-      lbias[i] = (valid && p.b_act) ? p.b_act[nid] : 0.f;
+      if (BIAS) lbias[i] = (valid && p.b_act) ? p.b_act[nid] : 0.f;
     }
   }
   __syncthreads();
@@ -199,22 +199,34 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 // ------------------------------------------ gathered FFN, 16-bit weights
 // Two phases per CTA, with no synchronisation inside either:
 //   up:   warp w computes the whole dot products of neurons w, w+8, ... of the
-//         slice (rows loaded with 128-bit loads straight into registers, x
-//         held in shared memory as fp32), reduces them within the warp and
-//         stores h in shared memory;
+//         slice: each row is read in passes of 32 x kPassChunks 16-byte chunks
+//         with 128-bit loads straight into registers, x is held in shared
+//         memory as fp32, the warp reduces the dot products and stores h in
+//         shared memory;
 //   down: after one CTA barrier, thread t owns the 16-byte column chunks
-//         t, t+256, ... of y and streams those chunks of every neuron's
-//         W_down^T row through registers (kDownRegs loads in flight),
-//         accumulating h * row into fp32 registers.
-// Every gathered row is read exactly once, in 512-byte warp-wide pieces.
+//         t, t+NT, ... of y and streams those chunks of every neuron's
+//         W_down^T row through registers, accumulating h * row in fp32.
+// Both phases are software-pipelined over two register buffers, so the next
+// tile's loads are always in flight while the current tile is consumed, and
+// the first loads of each phase are issued before the barrier that precedes
+// it.  Every gathered row is read exactly once, in 512-byte warp-wide pieces.
 // (Measured on B200: gathered 8 KB rows stream at about 6.1 TB/s through
-// registers this way; a shared-memory ring fed by one bulk-copy thread per
-// CTA reached about 5.4 TB/s with no work attached, and its per-neuron block
-// reductions and stage hand-offs held the real kernel near 3 TB/s.)
-constexpr int kLdgThreads = 256;
+// registers; a shared-memory ring fed by one bulk-copy thread per CTA reached
+// about 5.4 TB/s with no work attached, and L2 prefetching of the rows ahead
+// of use made this kernel slower.)
+#ifndef PI_LDG_THREADS
+#define PI_LDG_THREADS 256
+#endif
+#ifndef PI_PASS_CHUNKS
+#define PI_PASS_CHUNKS 8
+#endif
+#ifndef PI_DOWN_REGS
+#define PI_DOWN_REGS 8
+#endif
+constexpr int kLdgThreads = PI_LDG_THREADS;
 constexpr int kLdgWarps = kLdgThreads / 32;
-constexpr int kPassChunks = 16;  // up phase: 16-byte chunks per lane per pass
-constexpr int kDownRegs = 16;    // down phase: 16-byte loads in flight per thread
+constexpr int kPassChunks = PI_PASS_CHUNKS;  // up phase: chunks per lane per buffer
+constexpr int kDownRegs = PI_DOWN_REGS;      // down phase: 16-byte loads per thread per buffer
 
 // WDT: 0 fp16, 1 bf16 (activations of the same type).  ACT: 0 ReLU, 1 ReGLU.
 // CPT: down-phase column chunks per thread.  CPS: CTAs per SM.
@@ -224,10 +236,11 @@ __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
   constexpr int NUP = ACT == 1 ? 2 : 1;  // dot products per neuron
   constexpr int V = NUP * B;             // values reduced per neuron
   constexpr int SH = 5 - log2c<V>();
-  constexpr int D = kDownRegs / CPT > 0 ? kDownRegs / CPT : 1;  // down: neurons per batch
+  constexpr int PC = kPassChunks;
+  constexpr int DH = kDownRegs / CPT > 0 ? kDownRegs / CPT : 1;  // down: neurons per buffer
   int* scratch = reinterpret_cast<int*>(smem);                 // 64 ints
   int* ids = reinterpret_cast<int*>(smem + 256);               // [list_cap]
-  float* lbias = reinterpret_cast<float*>(ids + p.list_cap);   // [list_cap]
+  float* lbias = reinterpret_cast<float*>(ids + p.list_cap);   // [list_cap] (unused here)
   float* hs = lbias + p.list_cap;                              // [list_cap * B]
   float* xs = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(hs + (size_t)p.list_cap * B) + 15) & ~uintptr_t(15));  // [B*d]
@@ -235,11 +248,70 @@ __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
   pdl_trigger();
   pdl_wait();  // the list (or mask) and x come from earlier kernels
   int k0, k1;
-  build_slice<kLdgThreads>(p, scratch, ids, lbias, k0, k1);
+  build_slice<kLdgThreads, false>(p, scratch, ids, lbias, k0, k1);
   const int n = k1 - k0;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int d = p.d, nchunks = d / 8;
   const size_t rb = (size_t)d * 2;
+
+  // ------------------------------------------------------------- up phase
+  // This warp's work is a sequence of passes: neuron j (slice position
+  // warp + j * warps), matrix m (activation row, then W_up for ReGLU), pass k.
+  const int ppr = (nchunks + 32 * PC - 1) / (32 * PC);  // passes per row
+  const int my_n = warp < n ? (n - warp + kLdgWarps - 1) / kLdgWarps : 0;
+  const int P = my_n * NUP * ppr;
+  auto load_pass = [&](int pp, uint4 (&r)[PC]) {
+    const int j = pp / (NUP * ppr), rem = pp % (NUP * ppr);
+    const int m = rem / ppr, k = rem % ppr;
+    const int i = warp + j * kLdgWarps;
+    const int nid = ids[i] < 0 ? 0 : ids[i];
+    const uint8_t* row = (m == 0 ? p.w_act : p.w_up) + (size_t)nid * rb;
+#pragma unroll
+    for (int q = 0; q < PC; ++q) {
+      const int c = k * 32 * PC + lane + 32 * q;
+      r[q] = c < nchunks ? ldg_stream(row + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  float s[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) s[v] = 0.f;
+  float bias = 0.f;
+  auto consume_pass = [&](int pp, const uint4 (&r)[PC]) {
+    const int j = pp / (NUP * ppr), rem = pp % (NUP * ppr);
+    const int m = rem / ppr, k = rem % ppr;
+    const int i = warp + j * kLdgWarps;
+    if (rem == 0 && lane == 0) bias = (p.b_act && ids[i] >= 0) ? p.b_act[ids[i]] : 0.f;
+#pragma unroll
+    for (int q = 0; q < PC; ++q) {
+      const int c = k * 32 * PC + lane + 32 * q;
+      if (c < nchunks) {
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const float dv = dot8<WDT>(r[q], xs + (size_t)b * d + (size_t)c * 8);
+#pragma unroll
+          for (int mm = 0; mm < NUP; ++mm)
+            if (mm == m) s[mm * B + b] += dv;
+        }
+      }
+    }
+    if (rem == NUP * ppr - 1) {  // last pass of neuron i: reduce and store h
+      const float tot = warp_reduce_transposed<V>(s);
+      const int vi = lane >> SH;  // lane (v << SH) holds value v = m*B + b
+      float up = 1.f;
+      if constexpr (ACT == 1) up = __shfl_sync(0xffffffffu, tot, ((vi + B) % V) << SH);
+      const float bi = __shfl_sync(0xffffffffu, bias, 0);
+      if ((lane & ((1 << SH) - 1)) == 0 && vi < B) {
+        float h = fmaxf(tot + bi, 0.f);
+        if constexpr (ACT == 1) h *= up;
+        hs[(size_t)i * B + vi] = ids[i] < 0 ? 0.f : h;
+      }
+#pragma unroll
+      for (int v = 0; v < V; ++v) s[v] = 0.f;
+    }
+  };
+
+  uint4 ra[PC], rbuf[PC];
+  if (P > 0) load_pass(0, ra);  // in flight while x is staged
 
   for (int j = t; j < B * d / 8; j += kLdgThreads) {
     const uint4 v = *reinterpret_cast<const uint4*>(p.x + (size_t)j * 8);
@@ -247,59 +319,19 @@ __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
   }
   __syncthreads();
 
-  // ------------------------------------------------------------- up phase
-  for (int i = warp; i < n; i += kLdgWarps) {
-    const int nid = ids[i] < 0 ? 0 : ids[i];
-    float s[V];
-#pragma unroll
-    for (int v = 0; v < V; ++v) s[v] = 0.f;
-#pragma unroll
-    for (int m = 0; m < NUP; ++m) {
-      const uint8_t* row = (m == 0 ? p.w_act : p.w_up) + (size_t)nid * rb;
-      for (int c0 = 0; c0 < nchunks; c0 += 32 * kPassChunks) {
-        uint4 r[kPassChunks];
-#pragma unroll
-        for (int k = 0; k < kPassChunks; ++k) {
-          const int c = c0 + lane + 32 * k;
-          r[k] = c < nchunks ? ldg_stream(row + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int k = 0; k < kPassChunks; ++k) {
-          const int c = c0 + lane + 32 * k;
-          if (c < nchunks) {
-#pragma unroll
-            for (int b = 0; b < B; ++b)
-              s[m * B + b] += dot8<WDT>(r[k], xs + (size_t)b * d + (size_t)c * 8);
-          }
-        }
-      }
-    }
-    const float tot = warp_reduce_transposed<V>(s);
-    // lane (v << SH) holds value v = m*B + b; ReGLU fetches its up product
-    const int vi = lane >> SH;
-    float up = 1.f;
-    if constexpr (ACT == 1) up = __shfl_sync(0xffffffffu, tot, ((vi + B) % V) << SH);
-    if ((lane & ((1 << SH) - 1)) == 0 && vi < B) {
-      float h = fmaxf(tot + lbias[i], 0.f);
-      if constexpr (ACT == 1) h *= up;
-      hs[(size_t)i * B + vi] = ids[i] < 0 ? 0.f : h;
+  for (int pp = 0; pp < P; pp += 2) {
+    if (pp + 1 < P) load_pass(pp + 1, rbuf);
+    consume_pass(pp, ra);
+    if (pp + 1 < P) {
+      if (pp + 2 < P) load_pass(pp + 2, ra);
+      consume_pass(pp + 1, rbuf);
     }
   }
-  __syncthreads();
 
   // ----------------------------------------------------------- down phase
-  float acc[B][CPT][8];
+  auto load_down = [&](int i0, uint4 (&r)[DH][CPT]) {
 #pragma unroll
-  for (int b = 0; b < B; ++b)
-#pragma unroll
-    for (int c = 0; c < CPT; ++c)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[b][c][e] = 0.f;
-
-  for (int i0 = 0; i0 < n; i0 += D) {
-    uint4 r[D][CPT];
-#pragma unroll
-    for (int j = 0; j < D; ++j) {
+    for (int j = 0; j < DH; ++j) {
       const int i = i0 + j;
       const int nid = (i < n && ids[i] >= 0) ? ids[i] : 0;
       const uint8_t* row = p.w_dn + (size_t)nid * rb;
@@ -310,8 +342,17 @@ __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
                                          : make_uint4(0, 0, 0, 0);
       }
     }
+  };
+  float acc[B][CPT][8];
 #pragma unroll
-    for (int j = 0; j < D; ++j) {
+  for (int b = 0; b < B; ++b)
+#pragma unroll
+    for (int c = 0; c < CPT; ++c)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[b][c][e] = 0.f;
+  auto fma_down = [&](int i0, const uint4 (&r)[DH][CPT]) {
+#pragma unroll
+    for (int j = 0; j < DH; ++j) {
       const int i = i0 + j;
       if (i < n) {
         float hb[B];
@@ -331,6 +372,18 @@ __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
           }
         }
       }
+    }
+  };
+
+  uint4 d0[DH][CPT], d1[DH][CPT];
+  load_down(0, d0);  // in flight across the barrier (rows need no h)
+  __syncthreads();   // every h of the slice is in shared memory
+  for (int i0 = 0; i0 < n; i0 += 2 * DH) {
+    load_down(i0 + DH, d1);
+    fma_down(i0, d0);
+    if (i0 + DH < n) {
+      load_down(i0 + 2 * DH, d0);
+      fma_down(i0 + DH, d1);
     }
   }
 
@@ -585,32 +638,50 @@ __global__ void __launch_bounds__(32 * (NCW + 1), B == 1 ? 2 : 1) k_ffn_tma(FfnP
 }
 
 // ------------------------------------------------------ partial reduction
-// out[i] = sum over g = 0..G-1 (in this order within each of 8 slices, the
-// slices then added in order) of part[g][i]; MODE 0 writes y, MODE 1 adds into
-// the residual stream.  n4 = number of float4 columns (B*d/4).
+// out[i] = sum over g = 0..G-1 of part[g][i], MODE 0 writes y, MODE 1 adds into
+// the residual stream.  n4 = number of float4 columns (B*d/4).  A CTA covers 8
+// float4 columns with 32 slices each; slice s adds partials g = s, s+32, ...
+// in increasing g, and the 32 slice sums are then added in slice order, so the
+// summation order is fixed and y is reproducible.
+constexpr int kRedCols = 8;
+constexpr int kRedSlices = 32;
+
 template <int MODE>
-__global__ void __launch_bounds__(256) k_reduce(const float* __restrict__ part, int G, int n4,
-                                                float* __restrict__ out) {
-  __shared__ float4 sm[8][32];
+__global__ void __launch_bounds__(kRedCols * kRedSlices) k_reduce(const float* __restrict__ part,
+                                                                  int G, int n4,
+                                                                  float* __restrict__ out) {
+  __shared__ float4 sm[kRedSlices][kRedCols];
   pdl_wait();
   pdl_trigger();
-  const int col = blockIdx.x * 32 + (threadIdx.x & 31);
-  const int sl = threadIdx.x >> 5;
+  const int cl = threadIdx.x % kRedCols;
+  const int sl = threadIdx.x / kRedCols;
+  const int col = blockIdx.x * kRedCols + cl;
   float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
   if (col < n4) {
     const float4* src = reinterpret_cast<const float4*>(part);
-    for (int g = sl; g < G; g += 8) {
+    int g = sl;
+    for (; g + 3 * kRedSlices < G; g += 4 * kRedSlices) {
+      const float4 v0 = src[(size_t)g * n4 + col];
+      const float4 v1 = src[(size_t)(g + kRedSlices) * n4 + col];
+      const float4 v2 = src[(size_t)(g + 2 * kRedSlices) * n4 + col];
+      const float4 v3 = src[(size_t)(g + 3 * kRedSlices) * n4 + col];
+      t.x += v0.x; t.y += v0.y; t.z += v0.z; t.w += v0.w;
+      t.x += v1.x; t.y += v1.y; t.z += v1.z; t.w += v1.w;
+      t.x += v2.x; t.y += v2.y; t.z += v2.z; t.w += v2.w;
+      t.x += v3.x; t.y += v3.y; t.z += v3.z; t.w += v3.w;
+    }
+    for (; g < G; g += kRedSlices) {
       const float4 v = src[(size_t)g * n4 + col];
       t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
     }
   }
-  sm[sl][threadIdx.x & 31] = t;
+  sm[sl][cl] = t;
   __syncthreads();
   if (sl == 0 && col < n4) {
-    float4 r = sm[0][threadIdx.x];
+    float4 r = sm[0][cl];
 #pragma unroll
-    for (int k = 1; k < 8; ++k) {
-      const float4 v = sm[k][threadIdx.x];
+    for (int k = 1; k < kRedSlices; ++k) {
+      const float4 v = sm[k][cl];
       r.x += v.x; r.y += v.y; r.z += v.z; r.w += v.w;
     }
     float4* o = reinterpret_cast<float4*>(out) + col;

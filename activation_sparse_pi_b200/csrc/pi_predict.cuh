@@ -35,19 +35,33 @@ struct Pred1Params {
 
 // Layer input from the residual stream: x_l = round16(x / sqrt(mean(x^2) +
 // eps)) per token.  Every CTA computes it the same way (fixed summation
-// order), so all CTAs hold identical x_l.
+// order), so all CTAs hold identical x_l.  The residual is read once, with
+// 16-byte loads, and kept in registers between the reduction and the cast.
 template <int DT, int B>
 __device__ void rms_cast_to_smem(const float* __restrict__ xr, uint16_t* xs, int d,
                                  float* red /* >= [kConsumerWarps * B] */, uint16_t* x_out) {
+  // float4 per thread: d <= 8192 at B <= 2; the fused predictor takes B = 4 only for d <= 4096
+  constexpr int MAXV = (B == 4 ? 4096 : 8192) / (4 * kConsumers);
   const int ct = threadIdx.x - 32;
   const int lane = threadIdx.x & 31, w = ct >> 5;
+  const int n4 = d / 4;
+  float4 v[B][MAXV];
   float ss[B];
 #pragma unroll
   for (int b = 0; b < B; ++b) {
+#pragma unroll
+    for (int k = 0; k < MAXV; ++k) {
+      const int j = ct + kConsumers * k;
+      v[b][k] = j < n4 ? reinterpret_cast<const float4*>(xr + (size_t)b * d)[j]
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float t = 0.f;
-    for (int j = ct; j < d; j += kConsumers) {
-      float v = xr[(size_t)b * d + j];
-      t = fmaf(v, v, t);
+#pragma unroll
+    for (int k = 0; k < MAXV; ++k) {
+      t = fmaf(v[b][k].x, v[b][k].x, t);
+      t = fmaf(v[b][k].y, v[b][k].y, t);
+      t = fmaf(v[b][k].z, v[b][k].z, t);
+      t = fmaf(v[b][k].w, v[b][k].w, t);
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
@@ -63,10 +77,18 @@ __device__ void rms_cast_to_smem(const float* __restrict__ xr, uint16_t* xs, int
 #pragma unroll
     for (int i = 0; i < kConsumerWarps; ++i) t += red[i * B + b];
     const float rms = sqrtf(t / (float)d + kRmsEps);
-    for (int j = ct; j < d; j += kConsumers) {
-      uint16_t v = round16<DT>(xr[(size_t)b * d + j] / rms);
-      xs[(size_t)b * d + j] = v;
-      if (x_out) x_out[(size_t)b * d + j] = v;
+#pragma unroll
+    for (int k = 0; k < MAXV; ++k) {
+      const int j = ct + kConsumers * k;
+      if (j < n4) {
+        const uint32_t lo = (uint32_t)round16<DT>(v[b][k].x / rms) |
+                            ((uint32_t)round16<DT>(v[b][k].y / rms) << 16);
+        const uint32_t hi = (uint32_t)round16<DT>(v[b][k].z / rms) |
+                            ((uint32_t)round16<DT>(v[b][k].w / rms) << 16);
+        const uint2 pk = make_uint2(lo, hi);
+        reinterpret_cast<uint2*>(xs + (size_t)b * d)[j] = pk;
+        if (x_out) reinterpret_cast<uint2*>(x_out + (size_t)b * d)[j] = pk;
+      }
     }
   }
 }
@@ -244,6 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_pred2(Pred2Params p) {
   if (warp == 0) {
     if (lane == 0) {
       const uint8_t* base = p.w2 + (size_t)u0 * 32 * row_bytes;
+      // stages beyond the ring: ask the L2 for them now, while the previous
+      // kernel still runs, so the refills after the ring drains hit the L2
+      for (int i = NS; i < nst; ++i) prefetch_l2(base + (size_t)i * stage_bytes, stage_bytes);
       for (int i = 0; i < nst; ++i) {
         const int s = i % NS;
         if (i >= NS && !mbar_wait_sleep(&empty[s], ((i / NS) - 1) & 1)) break;
