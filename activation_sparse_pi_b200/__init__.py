@@ -27,6 +27,7 @@ from .binding import (  # noqa: F401
     pi_launch_count,
     pi_predict,
     pi_sparse_ffn,
+    pi_sparse_ffn_static,
     pi_status_string,
     pi_workspace_size,
     predictor_desc,

@@ -13,6 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libpi.so")
 
 PI_OK, PI_ERR_INVALID_ARG, PI_ERR_UNSUPPORTED, PI_ERR_WORKSPACE, PI_ERR_CUDA = range(5)
+PI_STATIC_SCRATCH_BYTES = 16 << 20  # fixed scratch of pi_sparse_ffn_static
 PI_F16, PI_BF16, PI_Q4_0 = 0, 1, 2
 PI_RELU, PI_REGLU = 0, 1
 DTYPES = {"f16": PI_F16, "bf16": PI_BF16, "q4_0": PI_Q4_0}
@@ -21,6 +22,7 @@ ACTS = {"relu": PI_RELU, "reglu": PI_REGLU}
 EXPORTS = (
     "pi_status_string", "pi_last_error", "pi_device_error", "pi_launch_count", "pi_workspace_size",
     "pi_predict", "pi_compact", "pi_sparse_ffn", "pi_ffn_stack", "pi_ffn_stack_timed",
+    "pi_sparse_ffn_static",
 )
 
 
@@ -78,6 +80,9 @@ def lib():
         L.pi_sparse_ffn.restype = c_int32
         L.pi_sparse_ffn.argtypes = [ctypes.POINTER(PiLayer), c_void_p, c_int32, c_void_p,
                                     c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
+        L.pi_sparse_ffn_static.restype = c_int32
+        L.pi_sparse_ffn_static.argtypes = [ctypes.POINTER(PiLayer), c_void_p, c_int32, c_void_p,
+                                           c_void_p, c_void_p, c_void_p]
         L.pi_ffn_stack.restype = c_int32
         L.pi_ffn_stack.argtypes = [ctypes.POINTER(PiLayer), c_int32, c_void_p, c_int32,
                                    c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
@@ -185,6 +190,12 @@ def pi_sparse_ffn(layer, x, batch, idx, count, y, workspace, stream=None):
     _check(lib().pi_sparse_ffn(ctypes.byref(layer), _ptr(x), int(batch), _ptr(idx), _ptr(count),
                                _ptr(y), _ptr(workspace), _nbytes(workspace), _stream(stream)),
            "pi_sparse_ffn")
+
+
+def pi_sparse_ffn_static(layer, x, batch, idx, count, y, stream=None):
+    _check(lib().pi_sparse_ffn_static(ctypes.byref(layer), _ptr(x), int(batch), _ptr(idx),
+                                      _ptr(count), _ptr(y), _stream(stream)),
+           "pi_sparse_ffn_static")
 
 
 def pi_ffn_stack(layers, x_resid, batch, idx_out, count_out, workspace, stream=None):

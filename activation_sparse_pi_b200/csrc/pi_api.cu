@@ -22,6 +22,12 @@
 
 using namespace pi;
 
+// Fixed device scratch of pi_sparse_ffn_static: the per-CTA partial sums of y
+// (and, on the batched path, the activations h).  It is part of the module
+// image, so the call never allocates; every device the library runs on
+// carries one copy, and concurrent calls on one device share it.
+static __device__ __align__(256) uint8_t g_static_scratch[PI_STATIC_SCRATCH_BYTES];
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -743,6 +749,61 @@ int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_re
       return s;
   }
   return PI_OK;
+}
+
+// Callers that cannot allocate -- a host framework whose allocator owns the
+// whole device, a latency-bound loop in which an allocation (which may wait
+// for the device) is not allowed, or code that only holds weights and
+// activations -- get the gathered FFN without supplying a workspace.
+// The scratch lives in g_static_scratch; its address is looked up once per
+// device (the first call on a device does this, so make it before any stream
+// capture).  Nothing in the scratch has to start at zero: every CTA writes its
+// whole partial plane, and h is written for every listed neuron before it is
+// read.  Calls whose work overlaps on one device race on the scratch.
+int32_t pi_sparse_ffn_static(const pi_layer* layer, const void* x, int32_t batch,
+                             const int32_t* idx, const int32_t* count, float* y, void* stream) {
+  if (int32_t s = validate_layer(layer)) return s;
+  if (int32_t s = validate_batch(batch)) return s;
+  if (!x || !idx || !count || !y) return fail(PI_ERR_INVALID_ARG, "x, idx, count and y are required");
+  if (!aligned16(x) || !aligned16(idx) || !aligned16(y) || (reinterpret_cast<uintptr_t>(count) & 3u))
+    return fail(PI_ERR_INVALID_ARG, "x, idx and y must be 16-byte aligned, count 4-byte aligned");
+  // the same scratch ffn_impl uses, packed from offset 0: partials, then h
+  const int d = layer->d_model;
+  const bool fused = ffn_fused_ok(layer, batch);
+  const int G = fused ? ffn_grid(batch) : down_slices(d, batch, num_sms());
+  WsLayout w{};
+  w.part = 0;
+  w.h = al256((size_t)G * batch * d * 4);
+  w.total = fused ? w.h : w.h + al256((size_t)layer->d_ff * batch * 4);
+  if (w.total > (size_t)PI_STATIC_SCRATCH_BYTES)
+    return fail(PI_ERR_WORKSPACE,
+                "pi_sparse_ffn_static: this shape needs %zu bytes of scratch, the fixed scratch "
+                "holds %zu; use pi_sparse_ffn with a workspace",
+                w.total, (size_t)PI_STATIC_SCRATCH_BYTES);
+  int dev = 0;
+  PI_CUDA(cudaGetDevice(&dev));
+  constexpr int kMaxDevices = 64;
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(PI_ERR_UNSUPPORTED, "device ordinal %d: the fixed scratch supports 0..%d", dev,
+                kMaxDevices - 1);
+  static std::mutex mu;
+  static uint8_t* base[kMaxDevices] = {};
+  uint8_t* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!base[dev]) {
+      void* ptr = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+      if (e != cudaSuccess)
+        return fail(PI_ERR_CUDA, "cudaGetSymbolAddress(fixed scratch) failed: %s",
+                    cudaGetErrorString(e));
+      base[dev] = static_cast<uint8_t*>(ptr);
+    }
+    ws = base[dev];
+  }
+  FfnSrc src{idx, count, nullptr, 0, nullptr, nullptr};
+  return ffn_impl(layer, batch, static_cast<const uint16_t*>(x), src, y, 0, w, ws,
+                  static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

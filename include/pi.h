@@ -174,6 +174,32 @@ int32_t pi_sparse_ffn(const pi_layer* layer, const void* x, int32_t batch,
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Size of the fixed device scratch that pi_sparse_ffn_static uses (16 MiB).
+ */
+#define PI_STATIC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * pi_sparse_ffn without a workspace argument.  This entry point has no
+ * counterpart in the pages the method is described on; it exists for callers
+ * that may not allocate device memory (an allocator owned by a host framework,
+ * a loop in which an allocation and the wait it can imply are not allowed).
+ * Arguments, layouts and results are those of pi_sparse_ffn, bit for bit.
+ * - Scratch: a PI_STATIC_SCRATCH_BYTES array in the library's own device
+ *   image, one per device.  The call allocates and frees nothing.
+ * - Limit: the call needs (CTA partials + on the batched path h) bytes of
+ *   scratch; pi_workspace_size(layer, 1, batch) <= PI_STATIC_SCRATCH_BYTES is
+ *   enough.  On a 148-SM device that covers every batch up to 6 at every
+ *   supported d_model and d_ff.  Larger shapes return PI_ERR_WORKSPACE
+ *   with the bytes needed and enqueue nothing.
+ * - Set-up: the first call on each device looks up the scratch address; make
+ *   it before any stream capture.
+ * - Concurrency: calls whose kernels may overlap on one device (different
+ *   streams, or host threads) race on the shared scratch; serialise them.
+ */
+int32_t pi_sparse_ffn_static(const pi_layer* layer, const void* x, int32_t batch,
+                             const int32_t* idx, const int32_t* count, float* y, void* stream);
+
+/*
  * Steps 1-4 over a stack of layers, for one batch of tokens.  For each layer
  * l: x_l = round16(x_resid / sqrt(mean(x_resid^2) + 1e-6)) per token (round
  * to nearest even into layer->adtype), then predict, compact and the gathered

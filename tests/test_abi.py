@@ -140,3 +140,26 @@ def test_compact_and_stack_validation(lib):
     assert st == pi.binding.PI_ERR_INVALID_ARG  # mixed d_model
     st = _status(pi.pi_ffn_stack, [L1], FAKE, 1, None, None, None)
     assert st == pi.binding.PI_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("d,B", [(4096, 8), (2048, 8), (8192, 64), (512, 64)])
+def test_static_scratch_rejects_oversized_shapes(lib, d, B):
+    # each shape needs more than the fixed scratch holds; the call must refuse
+    # before touching the device (only refused shapes may use fake pointers)
+    L = _layer(d_model=d, pred=_pred(d_model=d))
+    st = _status(pi.pi_sparse_ffn_static, L, FAKE, B, FAKE, FAKE, FAKE)
+    assert st == pi.binding.PI_ERR_WORKSPACE, pi.pi_last_error()
+    msg = pi.pi_last_error()
+    assert "needs" in msg and str(pi.binding.PI_STATIC_SCRATCH_BYTES) in msg, msg
+
+
+def test_static_scratch_validates_arguments(lib):
+    L = _layer()
+    st = _status(pi.pi_sparse_ffn_static, L, None, 1, FAKE, FAKE, FAKE)
+    assert st == pi.binding.PI_ERR_INVALID_ARG
+    st = _status(pi.pi_sparse_ffn_static, L, FAKE + 8, 1, FAKE, FAKE, FAKE)
+    assert st == pi.binding.PI_ERR_INVALID_ARG
+    st = _status(pi.pi_sparse_ffn_static, L, FAKE, 65, FAKE, FAKE, FAKE)
+    assert st == pi.binding.PI_ERR_UNSUPPORTED
+    st = _status(pi.pi_sparse_ffn_static, _layer(w_down_t=None), FAKE, 1, FAKE, FAKE, FAKE)
+    assert st == pi.binding.PI_ERR_INVALID_ARG
