@@ -69,7 +69,10 @@ int num_sms() {
 
 constexpr size_t kSmemMax = 227 * 1024;
 constexpr size_t kSmemPred1 = 96 * 1024;
-constexpr size_t kSmemPred2 = 160 * 1024;
+#ifndef PI_SMEM_PRED2_KB
+#define PI_SMEM_PRED2_KB 160
+#endif
+constexpr size_t kSmemPred2 = PI_SMEM_PRED2_KB * 1024;
 constexpr size_t kSmemFfn = 220 * 1024;  // shared by the CTAs on one SM
 constexpr size_t kPartCap = 64ull << 20;  // bytes of batched down partials
 
@@ -86,7 +89,7 @@ int ffn_grid(int B);
 
 // ------------------------------------------------------------ workspace
 struct WsLayout {
-  size_t a, mask, idx, count, xl, part, h, total;
+  size_t bar, a, mask, idx, count, xl, part, h, total;
 };
 
 int down_slices(int d, int B, int nsm) {
@@ -101,6 +104,7 @@ WsLayout ws_layout(int d, int F, int r, int B) {
   const int nsm = num_sms();
   WsLayout w{};
   size_t o = 0;
+  w.bar = o;   o += 256;
   w.a = o;     o += al256((size_t)B * r * 4);
   w.mask = o;  o += al256((size_t)B * (F / 32) * 4);
   w.idx = o;   o += al256((size_t)F * 4);
@@ -337,11 +341,98 @@ cudaError_t rows_bb(const RowsParams& p, int nrows_work, cudaStream_t st) {
   return launch_rows<DT, MODE, 64>(p, nrows_work, st);
 }
 
+// Both predictor layers in one kernel (batch 1-2): chunks per thread of a W1
+// row (CPT) and per lane of a W2 row (CPL).
+int pred_cpt(int d) {
+  const int need = (d / 8 + kPredThreads - 1) / kPredThreads;
+  for (int c : {1, 2, 4})
+    if (c >= need) return c;
+  return 0;
+}
+int pred_cpl(int r) {
+  const int need = (r / 8 + 31) / 32;
+  for (int c : {1, 2, 4, 8})
+    if (c >= need) return c;
+  return 0;
+}
+
+template <int DT, int B, int CPT, int CPL>
+cudaError_t launch_predict(const pi_predictor* P, const uint16_t* x, const float* xr,
+                           uint16_t* xo, float* a, uint32_t* mask, float* logits, uint32_t* bar,
+                           cudaStream_t st) {
+  auto kern = k_predict<DT, B, CPT, CPL>;
+  // every CTA must be resident at once for the grid barrier
+  int occ = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kPredThreads, 0);
+  if (e != cudaSuccess) return e;
+  // the grid barrier's ticket counter needs one grid size for every launch
+  if (occ < 2) return cudaErrorInvalidConfiguration;
+  const int G = num_sms() * 2;
+  if ((P->d_ff / 8 + G - 1) / G > kPredMaxUnits || (P->rank + G - 1) / G > kPredMaxRows1)
+    return cudaErrorInvalidValue;
+  PredParams p{};
+  p.w1 = static_cast<const uint8_t*>(P->w1);
+  p.b1 = P->b1;
+  p.x = x;
+  p.x_resid = xr;
+  p.x_out = xo;
+  p.a = a;
+  p.w2 = static_cast<const uint8_t*>(P->w2);
+  p.b2 = P->b2;
+  p.mask = reinterpret_cast<uint8_t*>(mask);
+  p.logits = logits;
+  p.bar = bar;
+  p.threshold = P->threshold;
+  p.d = P->d_model;
+  p.r = P->rank;
+  p.F = P->d_ff;
+  return launch(kern, dim3(G), dim3(kPredThreads), 0, st, p);
+}
+
+bool predict_fused_ok(int B, const pi_predictor* P) {
+  if (B != 1 && B != 2) return false;
+  const int cpt = pred_cpt(P->d_model), cpl = pred_cpl(P->rank);
+  if (cpt == 0 || cpl == 0 || B * cpt > 4 || B * cpl > 8) return false;
+  return (P->d_ff / 8 + num_sms() - 1) / num_sms() <= kPredMaxUnits &&
+         (P->rank + num_sms() - 1) / num_sms() <= kPredMaxRows1;
+}
+
+template <int DT, int B, int CPT>
+cudaError_t predict_cpl(const pi_predictor* P, const uint16_t* x, const float* xr, uint16_t* xo,
+                        float* a, uint32_t* mask, float* logits, uint32_t* bar, cudaStream_t st) {
+  switch (pred_cpl(P->rank)) {
+    case 1: return launch_predict<DT, B, CPT, 1>(P, x, xr, xo, a, mask, logits, bar, st);
+    case 2: return launch_predict<DT, B, CPT, 2>(P, x, xr, xo, a, mask, logits, bar, st);
+    case 4: return launch_predict<DT, B, CPT, 4>(P, x, xr, xo, a, mask, logits, bar, st);
+    case 8: if constexpr (B == 1) return launch_predict<DT, B, CPT, 8>(P, x, xr, xo, a, mask, logits, bar, st); break;
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int DT, int B>
+cudaError_t predict_cpt(const pi_predictor* P, const uint16_t* x, const float* xr, uint16_t* xo,
+                        float* a, uint32_t* mask, float* logits, uint32_t* bar, cudaStream_t st) {
+  switch (pred_cpt(P->d_model)) {
+    case 1: return predict_cpl<DT, B, 1>(P, x, xr, xo, a, mask, logits, bar, st);
+    case 2: return predict_cpl<DT, B, 2>(P, x, xr, xo, a, mask, logits, bar, st);
+    case 4: if constexpr (B == 1) return predict_cpl<DT, B, 4>(P, x, xr, xo, a, mask, logits, bar, st); break;
+  }
+  return cudaErrorInvalidValue;
+}
+
 // x16: 16-bit input, or null with xr (residual) given; xo receives x_l then.
+// bar: the workspace's grid-barrier words, zeroed by the API call beforehand.
 template <int DT>
 int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const float* xr,
-                     uint16_t* xo, uint32_t* mask, float* logits, float* a, cudaStream_t st) {
+                     uint16_t* xo, uint32_t* mask, float* logits, float* a, uint32_t* bar,
+                     cudaStream_t st) {
   const int d = P->d_model;
+  if (predict_fused_ok(B, P)) {
+    const cudaError_t e = B == 1 ? predict_cpt<DT, 1>(P, x16, xr, xo, a, mask, logits, bar, st)
+                                 : predict_cpt<DT, 2>(P, x16, xr, xo, a, mask, logits, bar, st);
+    if (e != cudaSuccess) return fail(PI_ERR_CUDA, "predictor launch failed: %s", cudaGetErrorString(e));
+    return PI_OK;
+  }
   if (pred1_fused_ok(B, d)) {
     PI_CUDA((pred1_dispatch<DT>(P, B, x16, xr, xo, a, st)));
   } else {
@@ -432,6 +523,8 @@ bool ffn_fused_ok(const pi_layer* L, int B) {
   }
   const int c = ldg_cpt(L->d_model);
   if (c == 0 || B * c > 8) return false;
+  // a warp's neurons: at most 64 (two bias registers per lane)
+  if ((ffn_list_cap(L, B) + kLdgWarps - 1) / kLdgWarps > 64) return false;
   return ldg_smem(L, B) <= kSmemFfn / ffn_cps(B);
 }
 
@@ -655,11 +748,13 @@ int32_t pi_predict(const pi_predictor* pred, const void* x, int32_t batch, uint3
   const WsLayout w = ws_layout(pred->d_model, pred->d_ff, pred->rank, batch);
   if (int32_t s = check_ws(workspace, workspace_bytes, w.a + (size_t)batch * pred->rank * 4)) return s;
   float* a = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.a);
+  uint32_t* bar = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + w.bar);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  PI_CUDA(cudaMemsetAsync(bar, 0, 8, st));
   const uint16_t* x16 = static_cast<const uint16_t*>(x);
   if (pred->dtype == PI_F16)
-    return predict_impl<0>(pred, batch, x16, nullptr, nullptr, mask_bits, logits, a, st);
-  return predict_impl<1>(pred, batch, x16, nullptr, nullptr, mask_bits, logits, a, st);
+    return predict_impl<0>(pred, batch, x16, nullptr, nullptr, mask_bits, logits, a, bar, st);
+  return predict_impl<1>(pred, batch, x16, nullptr, nullptr, mask_bits, logits, a, bar, st);
 }
 
 int32_t pi_compact(const uint32_t* mask_bits, int32_t batch, int32_t d_ff, int32_t* idx,
@@ -725,13 +820,15 @@ int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_re
   uint16_t* xl = reinterpret_cast<uint16_t*>(ws + w.xl);
   float* a = reinterpret_cast<float*>(ws + w.a);
   uint32_t* mask = reinterpret_cast<uint32_t*>(ws + w.mask);
+  uint32_t* bar = reinterpret_cast<uint32_t*>(ws + w.bar);
+  PI_CUDA(cudaMemsetAsync(bar, 0, 8, st));
   for (int l = 0; l < n_layers; ++l) {
     const pi_layer* L = &layers[l];
     int32_t* idx = idx_out ? idx_out + (size_t)l * L->d_ff : reinterpret_cast<int32_t*>(ws + w.idx);
     int32_t* cnt = count_out ? count_out + l : reinterpret_cast<int32_t*>(ws + w.count);
     int32_t s = (L->adtype == PI_F16)
-                    ? predict_impl<0>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, st)
-                    : predict_impl<1>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, st);
+                    ? predict_impl<0>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, bar, st)
+                    : predict_impl<1>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, bar, st);
     if (s) return s;
     if (ffn_events && (!ffn_events[2 * l] || !ffn_events[2 * l + 1]))
       return fail(PI_ERR_INVALID_ARG, "ffn_events[%d..%d] must be events", 2 * l, 2 * l + 1);

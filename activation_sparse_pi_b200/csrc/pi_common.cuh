@@ -19,8 +19,11 @@ constexpr uint32_t kWaitLimit = 1u << 22;
 // Suspend-hinted waits: each poll may sleep up to kSuspendNs before returning,
 // so a waiting warp does not spin; kWaitLimitSleep polls bound the wait to
 // about one second.
-constexpr uint32_t kSuspendNs = 2000;
-constexpr uint32_t kWaitLimitSleep = 1u << 19;
+#ifndef PI_SUSPEND_NS
+#define PI_SUSPEND_NS 2000
+#endif
+constexpr uint32_t kSuspendNs = PI_SUSPEND_NS;
+constexpr uint32_t kWaitLimitSleep = (1u << 19) * (2000u / (PI_SUSPEND_NS < 2000 ? PI_SUSPEND_NS : 2000));
 
 // Device error word (read and cleared by pi_device_error()).
 __device__ int g_dev_error;
@@ -184,6 +187,55 @@ __device__ __forceinline__ uint16_t round16(float v) {
 // mantissa bits of 2^23 and subtract 2^23 + 8.
 __device__ __forceinline__ float q4_val(uint32_t q) {
   return __uint_as_float(0x4B000000u | q) - 8388616.0f;
+}
+
+// ------------------------------------------------------- plain loads
+// 128-bit streaming load of read-only data (read once: no L1 allocation).
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// ------------------------------------------------------- grid barrier
+// Barrier over all CTAs of a grid whose CTAs are all resident at once (the
+// launcher sizes the grid from the occupancy calculator).  *count is a ticket
+// counter: it is 0 before the first barrier of an API call and every barrier
+// adds gridDim.x to it, so the k-th barrier (from 0) releases when it reaches
+// (k + 1) * gridDim.x.  Every grid that uses one counter between two zeroings
+// must have the same size.  The wait is bounded: on timeout the device error
+// word records kErrTimeout and the call returns false.
+constexpr uint32_t kGridWaitLimit = 1u << 21;  // about a second of polls
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ bool grid_barrier(uint32_t* count) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();  // this CTA's writes happen before its arrival
+    const uint32_t ticket = atomicAdd(count, 1u);
+    const uint32_t target = (ticket / gridDim.x + 1) * gridDim.x;
+    uint32_t it = 0;
+    while ((int32_t)(ld_acquire_gpu(count) - target) < 0) {
+      if (++it == kGridWaitLimit) {
+        set_error(kErrTimeout);
+        ok = 0;
+        break;
+      }
+      __nanosleep(32);
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
 }
 
 // ------------------------------------------------------- warp reductions

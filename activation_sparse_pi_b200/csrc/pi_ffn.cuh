@@ -187,14 +187,6 @@ __device__ void build_slice(const FfnParams& p, int* scratch, int* ids, float* l
   __syncthreads();
 }
 
-// 128-bit streaming load (read once: no L1 allocation).
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
 
 // ------------------------------------------ gathered FFN, 16-bit weights
 // Two phases per CTA, with no synchronisation inside either:
@@ -275,12 +267,18 @@ __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
   float s[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) s[v] = 0.f;
-  float bias = 0.f;
+  // biases of this warp's neurons, requested up front: lane l holds neuron
+  // l (and l + 32) of the warp's sequence, fetched by a shuffle when needed
+  float bias_lo = 0.f, bias_hi = 0.f;
+  if (p.b_act) {
+    const int i_lo = warp + lane * kLdgWarps, i_hi = warp + (lane + 32) * kLdgWarps;
+    if (lane < my_n && ids[i_lo] >= 0) bias_lo = p.b_act[ids[i_lo]];
+    if (lane + 32 < my_n && ids[i_hi] >= 0) bias_hi = p.b_act[ids[i_hi]];
+  }
   auto consume_pass = [&](int pp, const uint4 (&r)[PC]) {
     const int j = pp / (NUP * ppr), rem = pp % (NUP * ppr);
     const int m = rem / ppr, k = rem % ppr;
     const int i = warp + j * kLdgWarps;
-    if (rem == 0 && lane == 0) bias = (p.b_act && ids[i] >= 0) ? p.b_act[ids[i]] : 0.f;
 #pragma unroll
     for (int q = 0; q < PC; ++q) {
       const int c = k * 32 * PC + lane + 32 * q;
@@ -299,7 +297,7 @@ __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
       const int vi = lane >> SH;  // lane (v << SH) holds value v = m*B + b
       float up = 1.f;
       if constexpr (ACT == 1) up = __shfl_sync(0xffffffffu, tot, ((vi + B) % V) << SH);
-      const float bi = __shfl_sync(0xffffffffu, bias, 0);
+      const float bi = __shfl_sync(0xffffffffu, j < 32 ? bias_lo : bias_hi, j & 31);
       if ((lane & ((1 << SH) - 1)) == 0 && vi < B) {
         float h = fmaxf(tot + bi, 0.f);
         if constexpr (ACT == 1) h *= up;

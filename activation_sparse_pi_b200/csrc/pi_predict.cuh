@@ -357,4 +357,262 @@ __global__ void __launch_bounds__(kThreads, 1) k_pred2(Pred2Params p) {
   }
 }
 
+// ------------------------------------------------ both layers, one kernel
+// For batch 1-2 both predictor layers run in one grid of two CTAs per SM with
+// plain 128-bit register loads, split by a grid-wide barrier.
+//   Before the dependency wait: each CTA loads its first W1 rows into
+//   registers and asks the L2 for its W2 rows; none of this depends on the
+//   previous kernel.
+//   Layer 1: row j of W1 goes to CTA j mod G; all 256 threads share each row
+//   (thread t holds the 16-byte chunks t, t+256, ... of x and of the row); one
+//   block reduction per group of rows gives a_j = relu(W1_j x + b1_j).
+//   Grid barrier: every a_j is written.
+//   Layer 2: unit u (rows 8u..8u+7 of W2, one mask byte per token) goes to CTA
+//   u mod G; warp w of the CTA takes row 8u+w.  The eight bits of a unit meet
+//   in shared memory, and each mask byte is written once with a byte store.
+struct PredParams {
+  const uint8_t* w1;       // [r x d] 16-bit rows
+  const float* b1;         // [r] or null
+  const uint16_t* x;       // [B x d] 16-bit input (when x_resid is null)
+  const float* x_resid;    // [B x d] fp32 residual stream, or null
+  uint16_t* x_out;         // [B x d] rounded layer input (written when x_resid)
+  float* a;                // [B x r] fp32
+  const uint8_t* w2;       // [F x r] 16-bit rows
+  const float* b2;         // [F]
+  uint8_t* mask;           // [B x F/8] bytes: the uint32 mask words, byte-addressed
+  float* logits;           // [B x F] or null
+  uint32_t* bar;           // [2] grid barrier state
+  float threshold;
+  int d, r, F;
+};
+
+#ifndef PI_PRED_PF
+#define PI_PRED_PF 0
+#endif
+constexpr int kPredThreads = 256;
+constexpr int kPredWarps = kPredThreads / 32;
+constexpr int kPredMaxUnits = 64;  // units of 8 rows per CTA
+constexpr int kPredMaxRows1 = 32;  // W1 rows per CTA
+
+__host__ __device__ constexpr int pred_p2(int B, int CPL) {
+  // layer-2 units in flight per warp: about 96 registers for a and the rows
+  return (96 - 8 * B * CPL) / (4 * CPL) < 1 ? 1
+         : (96 - 8 * B * CPL) / (4 * CPL) > 8 ? 8
+                                               : (96 - 8 * B * CPL) / (4 * CPL);
+}
+
+template <int DT, int B, int CPT, int CPL>
+__global__ void __launch_bounds__(kPredThreads, 2) k_predict(PredParams p) {
+  constexpr int P1 = 8 / CPT;        // W1 rows in flight per thread
+  constexpr int V1 = P1 * B;
+  constexpr int SH1 = 5 - log2c<V1>();
+  constexpr int P2 = pred_p2(B, CPL);
+  static_assert(B * CPT <= 4 && B * CPL <= 8, "register budget");
+  __shared__ float red1[2][kPredWarps][V1];
+  __shared__ float redx[kPredWarps][B];
+  __shared__ uint32_t bits[B][kPredMaxUnits];
+  __shared__ float bias1[kPredMaxRows1];
+  __shared__ float bias2[kPredMaxUnits][kPredWarps];
+
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int nch1 = p.d / 8;
+  const size_t rb1 = (size_t)p.d * 2;
+  const int n1 = c < p.r ? (p.r - 1 - c) / G + 1 : 0;  // W1 rows c, c+G, ...
+  const int nunits = p.F / 8;
+  const int n2 = c < nunits ? (nunits - 1 - c) / G + 1 : 0;  // W2 units c, c+G, ...
+  const int nch2 = p.r / 8;
+  const size_t rb2 = (size_t)p.r * 2;
+
+  auto load1 = [&](int i, uint4 (&dst)[CPT]) {
+    const uint8_t* row = p.w1 + (size_t)(c + i * G) * rb1;
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+      const int u = t + kPredThreads * k;
+      dst[k] = (i < n1 && u < nch1) ? ldg_stream(row + (size_t)u * 16) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  uint4 wb[P1][CPT];
+#pragma unroll
+  for (int q = 0; q < P1; ++q) load1(q, wb[q]);
+
+  for (int e = t; e < B * kPredMaxUnits; e += kPredThreads) (&bits[0][0])[e] = 0u;
+  // static biases of this CTA's rows, off the critical path
+  if (t < n1) bias1[t] = p.b1 ? p.b1[c + t * G] : 0.f;
+  for (int e = t; e < n2 * 8; e += kPredThreads) bias2[e >> 3][e & 7] = p.b2[(size_t)(c + (e >> 3) * G) * 8 + (e & 7)];
+#if PI_PRED_PF == 1
+  if (t < n2) prefetch_l2(p.w2 + (size_t)(c + t * G) * 8 * rb2, (uint32_t)(8 * rb2));
+#endif
+
+  pdl_trigger();
+  pdl_wait();  // x (or the residual) comes from the previous kernel
+
+  // this thread's chunks of the layer input, widened to fp32
+  float xr[B][CPT][8];
+  if (p.x_resid) {
+    // x_l = round16(x / sqrt(mean(x^2) + eps)); every CTA forms the same sums
+    float4 v[B][CPT][2];
+    float ss[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      float s2 = 0.f;
+#pragma unroll
+      for (int k = 0; k < CPT; ++k) {
+        const int u = t + kPredThreads * k;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          v[b][k][h] = u < nch1 ? reinterpret_cast<const float4*>(p.x_resid + (size_t)b * p.d)[2 * u + h]
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+          s2 = fmaf(v[b][k][h].x, v[b][k][h].x, s2);
+          s2 = fmaf(v[b][k][h].y, v[b][k][h].y, s2);
+          s2 = fmaf(v[b][k][h].z, v[b][k][h].z, s2);
+          s2 = fmaf(v[b][k][h].w, v[b][k][h].w, s2);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+      ss[b] = s2;
+    }
+    if (lane == 0)
+#pragma unroll
+      for (int b = 0; b < B; ++b) redx[w][b] = ss[b];
+    __syncthreads();
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      float tot = 0.f;
+#pragma unroll
+      for (int i = 0; i < kPredWarps; ++i) tot += redx[i][b];
+      const float rms = sqrtf(tot / (float)p.d + kRmsEps);
+#pragma unroll
+      for (int k = 0; k < CPT; ++k) {
+        const int u = t + kPredThreads * k;
+        const float f[8] = {v[b][k][0].x, v[b][k][0].y, v[b][k][0].z, v[b][k][0].w,
+                            v[b][k][1].x, v[b][k][1].y, v[b][k][1].z, v[b][k][1].w};
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          pk[e] = (uint32_t)round16<DT>(f[2 * e] / rms) | ((uint32_t)round16<DT>(f[2 * e + 1] / rms) << 16);
+        const uint4 q4 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        if (u < nch1 && c == 0 && p.x_out)
+          reinterpret_cast<uint4*>(p.x_out + (size_t)b * p.d)[u] = q4;
+        widen8<DT>(u < nch1 ? q4 : make_uint4(0, 0, 0, 0), xr[b][k]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int b = 0; b < B; ++b)
+#pragma unroll
+      for (int k = 0; k < CPT; ++k) {
+        const int u = t + kPredThreads * k;
+        const uint4 q4 = u < nch1 ? reinterpret_cast<const uint4*>(p.x + (size_t)b * p.d)[u]
+                                  : make_uint4(0, 0, 0, 0);
+        widen8<DT>(q4, xr[b][k]);
+      }
+  }
+
+  // ---- layer 1
+  for (int base = 0; base < n1; base += P1) {
+    float v[V1];
+#pragma unroll
+    for (int q = 0; q < P1; ++q) {
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        float z = 0.f;
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) z += dot8<DT>(wb[q][k], xr[b][k]);
+        v[q * B + b] = z;
+      }
+      load1(base + q + P1, wb[q]);
+    }
+    const float tot = warp_reduce_transposed<V1>(v);
+    const int buf = (base / P1) & 1;
+    if ((lane & ((1 << SH1) - 1)) == 0) red1[buf][w][lane >> SH1] = tot;
+    __syncthreads();
+    if (t < V1) {
+      const int q = t / B, b = t % B, i = base + q;
+      if (i < n1) {
+        float z = 0.f;
+#pragma unroll
+        for (int k = 0; k < kPredWarps; ++k) z += red1[buf][k][t];
+        z += bias1[i];
+        p.a[(size_t)b * p.r + c + i * G] = fmaxf(z, 0.f);
+      }
+    }
+  }
+
+  // ---- layer 2: the first rows are requested before the barrier
+  auto load2 = [&](int i, uint4 (&dst)[CPL]) {
+    const uint8_t* row = p.w2 + ((size_t)(c + i * G) * 8 + w) * rb2;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+      const int cc = lane + 32 * k;
+      dst[k] = (i < n2 && cc < nch2) ? ldg_stream(row + (size_t)cc * 16) : make_uint4(0, 0, 0, 0);
+    }
+  };
+#if PI_PRED_PF == 2
+  if (t < n2) prefetch_l2(p.w2 + (size_t)(c + t * G) * 8 * rb2, (uint32_t)(8 * rb2));
+#endif
+  uint4 wr[P2][CPL];
+#pragma unroll
+  for (int q = 0; q < P2; ++q) load2(q, wr[q]);
+
+  const bool synced = grid_barrier(p.bar);
+
+  float av[B][CPL][8];
+#pragma unroll
+  for (int b = 0; b < B; ++b)
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+      const int cc = lane + 32 * k;
+      const float4* src = reinterpret_cast<const float4*>(p.a + (size_t)b * p.r) + 2 * cc;
+      const float4 lo = cc < nch2 ? __ldcg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 hi = cc < nch2 ? __ldcg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+      av[b][k][0] = lo.x; av[b][k][1] = lo.y; av[b][k][2] = lo.z; av[b][k][3] = lo.w;
+      av[b][k][4] = hi.x; av[b][k][5] = hi.y; av[b][k][6] = hi.z; av[b][k][7] = hi.w;
+    }
+
+  for (int base = 0; base < n2; base += P2) {
+#pragma unroll
+    for (int q = 0; q < P2; ++q) {
+      const int i = base + q;
+      float v[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b) v[b] = 0.f;
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) {
+        const uint32_t wv[4] = {wr[q][k].x, wr[q][k].y, wr[q][k].z, wr[q][k].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack2<DT>(wv[e]);
+#pragma unroll
+          for (int b = 0; b < B; ++b) {
+            v[b] = fmaf(f.x, av[b][k][2 * e], v[b]);
+            v[b] = fmaf(f.y, av[b][k][2 * e + 1], v[b]);
+          }
+        }
+      }
+      load2(i + P2, wr[q]);
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) v[b] += __shfl_xor_sync(0xffffffffu, v[b], o);
+      if (i < n2 && lane == 0 && synced) {
+        const int row = (c + i * G) * 8 + w;
+        const float bias = bias2[i][w];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const float s = v[b] + bias;
+          if (p.logits) p.logits[(size_t)b * p.F + row] = s;
+          if (s > p.threshold) atomicOr(&bits[b][i], 1u << w);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = t; e < B * n2; e += kPredThreads) {
+    const int b = e / n2, i = e % n2;
+    p.mask[(size_t)b * nunits + c + i * G] = (uint8_t)bits[b][i];
+  }
+}
+
 }  // namespace pi

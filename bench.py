@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip dense, mode F, e2e and CPU baseline legs")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--counts-out", default="",
+                    help="write the active-neuron count and algorithmic bytes of every "
+                         "gathered-FFN launch of one step (token x layer) as JSON")
     return ap.parse_args()
 
 
@@ -369,6 +372,11 @@ def run_ours(args, rank, world, local):
              "frac": round(stack_gbs / peak, 4), "bytes_per_step": round(stack_bytes),
              "timed_graph_step_ms": round(timed_step_ms, 3)}
     del gt, evs
+    if args.counts_out and rank == 0:
+        with open(args.counts_out, "w") as f:
+            json.dump({"order": "token-major, then layer", "counts": Ks.tolist(),
+                       "algorithmic_bytes": ffn_bytes.tolist(),
+                       "event_us": (durs * 1e3).round(3).tolist()}, f)
 
     extras = {}
     if not args.no_extras:
