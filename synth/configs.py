@@ -1,10 +1,10 @@
 """The five synthetic layer-stack workloads.
 
 Shapes follow the models the PowerInfer pages evaluate (OPT-6.7B,
-ReLU-Llama-2-13B, Falcon(ReLU)-40B, LLaMA(ReGLU)-70B; page 4, "Experiments",
-and page 3, "Model Weights" tables) plus one toy layer.  Activation fractions
-follow page 4's Figure 10 discussion (about 20% of neurons active per token for
-OPT-30B) and the workload descriptions these configs were specified with.
+ReLU-Llama-2-13B, Falcon(ReLU)-40B, LLaMA(ReGLU)-70B; the machine-heart page,
+experiments section, and the PyTorchKR page, "Model Weights" tables) plus one
+toy layer.  Activation fractions follow the machine-heart page's discussion of
+Figure 10 (about 20% of neurons active per token for OPT-30B).
 """
 from dataclasses import dataclass, field
 from typing import Tuple

@@ -12,8 +12,8 @@ Recipe (one layer, d = d_model, F = d_ff, r = predictor rank):
   to Q4_0 (blocks of 32 values with one fp16 scale) for the INT4 config.
 * Firing profile: a seeded permutation pi of the neurons and
   p_pi(k) = min(1, c k^-s), c bisected so the mean equals the target, clipped to
-  [1e-6, 1 - 1e-6] (page 1 and page 2 describe a power-law activation
-  distribution with a few "hot" neurons).
+  [1e-6, 1 - 1e-6] (the GeekNews page and the unite.ai page describe a
+  power-law activation distribution with a few "hot" neurons).
 * Bias of the activation row (b_up for ReLU, b_gate for ReGLU): layer inputs
   have unit RMS, so the pre-activation w_i . x + b_i is close to
   N(b_i, |w_i|^2) and b_i = |w_i| Phi^-1(p_i) gives firing probability p_i.
