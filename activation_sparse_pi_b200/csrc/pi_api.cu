@@ -118,29 +118,34 @@ WsLayout ws_layout(int d, int F, int r, int B) {
 }
 
 // ------------------------------------------------------------ launching
+cudaError_t allow_large_smem(const void* kern) {
+  // once per (device, kernel): allow the large dynamic shared memory carve-out
+  static std::mutex mu;
+  static std::set<std::pair<int, const void*>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const auto key = std::make_pair(dev, kern);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done.count(key)) {
+    // the carve-out is shared with the kernel's static shared memory
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(kSmemMax - fa.sharedSizeBytes));
+    if (e != cudaSuccess) return e;
+    done.insert(key);
+  }
+  return cudaSuccess;
+}
+
 template <typename Kern, typename... Args>
 cudaError_t launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                    Args... args) {
   if (smem > 48 * 1024) {
-    // once per (device, kernel): allow the large dynamic shared memory carve-out
-    static std::mutex mu;
-    static std::set<std::pair<int, const void*>> done;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    const cudaError_t e = allow_large_smem(reinterpret_cast<const void*>(kern));
     if (e != cudaSuccess) return e;
-    const auto key = std::make_pair(dev, reinterpret_cast<const void*>(kern));
-    std::lock_guard<std::mutex> lock(mu);
-    if (!done.count(key)) {
-      // the carve-out is shared with the kernel's static shared memory
-      cudaFuncAttributes fa{};
-      e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kern));
-      if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)(kSmemMax - fa.sharedSizeBytes));
-      if (e != cudaSuccess) return e;
-      done.insert(key);
-    }
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -492,7 +497,7 @@ int ldg_cpt(int d) {
 }
 
 size_t ldg_smem(const pi_layer* L, int B) {
-  return 256 + (size_t)ffn_list_cap(L, B) * (8 + 4 * B) + 16 + (size_t)B * L->d_model * 4;
+  return 256 + (size_t)ffn_list_cap(L, B) * (8 + 4 * B) + (size_t)L->d_ff / 4 + 16;
 }
 
 // Q4_0 weights (k_ffn_tma): 8 consumer warps, kTmaLanes producer lanes
@@ -502,7 +507,7 @@ constexpr int kTmaLanes = 2;
 size_t tma_fixed_smem(const pi_layer* L, int B) {
   const int V = kGroup * (L->act == PI_REGLU ? 2 : 1) * B;
   return 1024 + (size_t)ffn_list_cap(L, B) * 8 + (size_t)2 * kTmaNcw * V * 4 +
-         (size_t)2 * kGroup * B * 4 + 128;
+         (size_t)2 * kGroup * B * 4 + (size_t)L->d_ff / 4 + 128;
 }
 
 int tma_nstages(const pi_layer* L, int B) {
@@ -523,8 +528,6 @@ bool ffn_fused_ok(const pi_layer* L, int B) {
   }
   const int c = ldg_cpt(L->d_model);
   if (c == 0 || B * c > 8) return false;
-  // a warp's neurons: at most 64 (two bias registers per lane)
-  if ((ffn_list_cap(L, B) + kLdgWarps - 1) / kLdgWarps > 64) return false;
   return ldg_smem(L, B) <= kSmemFfn / ffn_cps(B);
 }
 
@@ -535,6 +538,7 @@ struct FfnSrc {            // where the fused kernel takes its neuron list from
   int mask_rows;
   int32_t* idx_out;        // mask mode: write the ascending list / count here
   int32_t* count_out;
+  const pi_predictor* next;  // predictor the stream runs next (L2 prefetch), or null
 };
 
 FfnParams ffn_params(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, float* part) {
@@ -556,6 +560,13 @@ FfnParams ffn_params(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& 
   p.F = L->d_ff;
   p.row_bytes = (uint32_t)ffn_row_bytes(L);
   p.list_cap = ffn_list_cap(L, B);
+  if (src.next) {
+    const pi_predictor* N = src.next;
+    p.pf_base[0] = static_cast<const uint8_t*>(N->w1);
+    p.pf_bytes[0] = (size_t)N->rank * N->d_model * 2;
+    p.pf_base[1] = static_cast<const uint8_t*>(N->w2);
+    p.pf_bytes[1] = (size_t)N->d_ff * N->rank * 2;
+  }
   return p;
 }
 
@@ -836,7 +847,7 @@ int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_re
     if (ffn_fused_ok(L, batch)) {
       // compaction fused into the FFN kernel: it reads the mask bits directly
       src = FfnSrc{nullptr, nullptr, mask, (int)batch, idx_out ? idx : nullptr,
-                   count_out ? cnt : nullptr};
+                   count_out ? cnt : nullptr, &layers[(l + 1) % n_layers].pred};
     } else {
       PI_CUDA((launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, (const uint32_t*)mask,
                       (int)batch, L->d_ff, idx, cnt)));

@@ -199,6 +199,30 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
+// The same load with an L2 eviction-priority policy (from createpolicy).
+__device__ __forceinline__ uint4 ldg_stream_hint(const void* p, uint64_t policy) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(policy));
+  return v;
+}
+
+// Ask the L2 for this CTA's share of a byte range (16-byte aligned start and
+// size): bytes [cta * share, (cta + 1) * share), in pieces of at most 32 KB.
+__device__ __forceinline__ void prefetch_l2_share(const uint8_t* base, size_t bytes, int cta,
+                                                  int nctas) {
+  if (!base || bytes == 0) return;
+  const size_t share = ((bytes + nctas - 1) / nctas + 15) & ~size_t(15);
+  const size_t lo = (size_t)cta * share;
+  if (lo >= bytes) return;
+  const size_t hi = lo + share < bytes ? lo + share : bytes;
+  for (size_t o = lo; o < hi; o += 32768) {
+    const size_t n = hi - o < 32768 ? hi - o : 32768;
+    prefetch_l2(base + o, (uint32_t)n);
+  }
+}
+
 // ------------------------------------------------------- grid barrier
 // Barrier over all CTAs of a grid whose CTAs are all resident at once (the
 // launcher sizes the grid from the occupancy calculator).  *count is a ticket

@@ -99,6 +99,10 @@ struct FfnParams {
   uint32_t row_bytes;
   int nstages;             // TMA kernel: ring stages
   int list_cap;
+  // weights the next kernels will read (the next layer's predictor), asked
+  // of the L2 while this kernel's prologue leaves DRAM idle; null for none
+  const uint8_t* pf_base[2];
+  size_t pf_bytes[2];
 };
 
 // Block-wide exclusive scan of one int per thread (all NT threads of the CTA).
@@ -133,8 +137,8 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch /* >= 33 ints
 // of invalid explicit entries are -1).  All NT threads call it; it ends with a
 // CTA barrier.
 template <int NT, bool BIAS = true>
-__device__ void build_slice(const FfnParams& p, int* scratch, int* ids, float* lbias, int& k0,
-                            int& k1) {
+__device__ void build_slice(const FfnParams& p, int* scratch, uint32_t* wbuf /* [2 x F/32] */,
+                            int* ids, float* lbias, int& k0, int& k1) {
   const int G = gridDim.x;
   if (p.mask) {
     const int W = p.F / 32;
@@ -157,19 +161,32 @@ __device__ void build_slice(const FfnParams& p, int* scratch, int* ids, float* l
     k0 = (int)(((long long)K * blockIdx.x) / G);
     k1 = (int)(((long long)K * (blockIdx.x + 1)) / G);
     if (blockIdx.x == 0 && threadIdx.x == 0 && p.count_out) *p.count_out = K;
+    // per-word exclusive prefix counts and the words themselves ...
+    uint32_t* wmask = wbuf;
+    int* wpre = reinterpret_cast<int*>(wbuf + W);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      uint32_t m = words[k];
-      while (m) {
-        const int nid = (w0 + k) * 32 + __ffs(m) - 1;
-        m &= m - 1;
-        if (pos >= k0 && pos < k1) {
-          ids[pos - k0] = nid;
-          if (BIAS) lbias[pos - k0] = p.b_act ? p.b_act[nid] : 0.f;
-          if (p.idx_out) p.idx_out[pos] = nid;
-        }
-        ++pos;
+      if (k < wpt && w0 + k < W) {
+        wmask[w0 + k] = words[k];
+        wpre[w0 + k] = pos;
+        pos += __popc(words[k]);
       }
+    }
+    __syncthreads();
+    // ... so that slice position i (rank k0 + i of the union) is found in
+    // parallel: its word by binary search, then its bit within the word
+    for (int i = threadIdx.x; i < k1 - k0; i += NT) {
+      const int q = k0 + i;
+      int lo = 0, hi = W - 1;  // the last word whose prefix is <= q
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (wpre[mid] <= q) lo = mid;
+        else hi = mid - 1;
+      }
+      const int nid = lo * 32 + (int)__fns(wmask[lo], 0, q - wpre[lo] + 1);
+      ids[i] = nid;
+      if (BIAS) lbias[i] = p.b_act ? p.b_act[nid] : 0.f;
+      if (p.idx_out) p.idx_out[q] = nid;
     }
   } else {
     int K = *p.count;
@@ -189,19 +206,20 @@ __device__ void build_slice(const FfnParams& p, int* scratch, int* ids, float* l
 
 
 // ------------------------------------------ gathered FFN, 16-bit weights
-// Two phases per CTA, with no synchronisation inside either:
-//   up:   warp w computes the whole dot products of neurons w, w+8, ... of the
-//         slice: each row is read in passes of 32 x kPassChunks 16-byte chunks
-//         with 128-bit loads straight into registers, x is held in shared
-//         memory as fp32, the warp reduces the dot products and stores h in
-//         shared memory;
+// Two phases per CTA over its slice of the neuron list:
+//   up:   the whole CTA works on every neuron, a group of R neurons at a time:
+//         thread t holds the 16-byte chunks t, t+NT, ... of x (fp32, in
+//         registers) and loads the same chunks of each of the group's rows
+//         with 128-bit loads straight into registers, so every row is
+//         requested whole and at once.  One block reduction per group gives
+//         the group's h, stored in shared memory;
 //   down: after one CTA barrier, thread t owns the 16-byte column chunks
 //         t, t+NT, ... of y and streams those chunks of every neuron's
 //         W_down^T row through registers, accumulating h * row in fp32.
 // Both phases are software-pipelined over two register buffers, so the next
-// tile's loads are always in flight while the current tile is consumed, and
+// group's loads are always in flight while the current one is consumed, and
 // the first loads of each phase are issued before the barrier that precedes
-// it.  Every gathered row is read exactly once, in 512-byte warp-wide pieces.
+// it.  Every gathered row is read exactly once.
 // (Measured on B200: gathered 8 KB rows stream at about 6.1 TB/s through
 // registers; a shared-memory ring fed by one bulk-copy thread per CTA reached
 // about 5.4 TB/s with no work attached, and L2 prefetching of the rows ahead
@@ -209,120 +227,135 @@ __device__ void build_slice(const FfnParams& p, int* scratch, int* ids, float* l
 #ifndef PI_LDG_THREADS
 #define PI_LDG_THREADS 256
 #endif
-#ifndef PI_PASS_CHUNKS
-#define PI_PASS_CHUNKS 8
+#ifndef PI_UP_REGS
+#define PI_UP_REGS 8
 #endif
 #ifndef PI_DOWN_REGS
 #define PI_DOWN_REGS 8
 #endif
 constexpr int kLdgThreads = PI_LDG_THREADS;
 constexpr int kLdgWarps = kLdgThreads / 32;
-constexpr int kPassChunks = PI_PASS_CHUNKS;  // up phase: chunks per lane per buffer
-constexpr int kDownRegs = PI_DOWN_REGS;      // down phase: 16-byte loads per thread per buffer
+constexpr int kUpRegs = PI_UP_REGS;      // up phase: 16-byte loads per thread per buffer
+constexpr int kDownRegs = PI_DOWN_REGS;  // down phase: 16-byte loads per thread per buffer
 
 // WDT: 0 fp16, 1 bf16 (activations of the same type).  ACT: 0 ReLU, 1 ReGLU.
-// CPT: down-phase column chunks per thread.  CPS: CTAs per SM.
+// CPT: column chunks per thread.  CPS: CTAs per SM.
 template <int WDT, int ACT, int B, int CPT, int CPS>
 __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int NUP = ACT == 1 ? 2 : 1;  // dot products per neuron
-  constexpr int V = NUP * B;             // values reduced per neuron
-  constexpr int SH = 5 - log2c<V>();
-  constexpr int PC = kPassChunks;
+  constexpr int NUP = ACT == 1 ? 2 : 1;  // rows per neuron in the up phase
+  constexpr int R = kUpRegs / (NUP * CPT) > 0 ? kUpRegs / (NUP * CPT) : 1;  // neurons per group
+  constexpr int VG = R * NUP * B;        // dot products per group
+  constexpr int SHG = 5 - log2c<VG>();
+  static_assert(VG <= 32 && (VG & (VG - 1)) == 0, "a group's dot products fit one warp reduction");
   constexpr int DH = kDownRegs / CPT > 0 ? kDownRegs / CPT : 1;  // down: neurons per buffer
   int* scratch = reinterpret_cast<int*>(smem);                 // 64 ints
   int* ids = reinterpret_cast<int*>(smem + 256);               // [list_cap]
-  float* lbias = reinterpret_cast<float*>(ids + p.list_cap);   // [list_cap] (unused here)
+  float* lbias = reinterpret_cast<float*>(ids + p.list_cap);   // [list_cap]
   float* hs = lbias + p.list_cap;                              // [list_cap * B]
-  float* xs = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(hs + (size_t)p.list_cap * B) + 15) & ~uintptr_t(15));  // [B*d]
+  uint32_t* wbuf = reinterpret_cast<uint32_t*>(hs + (size_t)p.list_cap * B);  // [2 x F/32]
+  __shared__ float red[2][kLdgWarps][VG];
 
-  pdl_trigger();
-  pdl_wait();  // the list (or mask) and x come from earlier kernels
-  int k0, k1;
-  build_slice<kLdgThreads, false>(p, scratch, ids, lbias, k0, k1);
-  const int n = k1 - k0;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int d = p.d, nchunks = d / 8;
   const size_t rb = (size_t)d * 2;
+  // gathered rows are read once: first in line for eviction from the L2, so
+  // that the prefetched weights below stay there
+  const uint64_t pol = policy_evict_first();
+#ifndef PI_FFN_PF
+#define PI_FFN_PF 1
+#endif
+  if (PI_FFN_PF && t == 0) {
+    prefetch_l2_share(p.pf_base[0], p.pf_bytes[0], blockIdx.x, gridDim.x);
+    prefetch_l2_share(p.pf_base[1], p.pf_bytes[1], blockIdx.x, gridDim.x);
+  }
+
+  pdl_trigger();
+  pdl_wait();  // the list (or mask) and x come from earlier kernels
+  // this thread's chunks of x, requested together with the mask words
+  uint4 xq[B][CPT];
+#pragma unroll
+  for (int b = 0; b < B; ++b)
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+      const int u = t + kLdgThreads * c;
+      xq[b][c] = u < nchunks ? reinterpret_cast<const uint4*>(p.x + (size_t)b * d)[u]
+                             : make_uint4(0, 0, 0, 0);
+    }
+  int k0, k1;
+  build_slice<kLdgThreads, false>(p, scratch, wbuf, ids, lbias, k0, k1);
+  const int n = k1 - k0;
 
   // ------------------------------------------------------------- up phase
-  // This warp's work is a sequence of passes: neuron j (slice position
-  // warp + j * warps), matrix m (activation row, then W_up for ReGLU), pass k.
-  const int ppr = (nchunks + 32 * PC - 1) / (32 * PC);  // passes per row
-  const int my_n = warp < n ? (n - warp + kLdgWarps - 1) / kLdgWarps : 0;
-  const int P = my_n * NUP * ppr;
-  auto load_pass = [&](int pp, uint4 (&r)[PC]) {
-    const int j = pp / (NUP * ppr), rem = pp % (NUP * ppr);
-    const int m = rem / ppr, k = rem % ppr;
-    const int i = warp + j * kLdgWarps;
-    const int nid = ids[i] < 0 ? 0 : ids[i];
-    const uint8_t* row = (m == 0 ? p.w_act : p.w_up) + (size_t)nid * rb;
+  const int ngroups = (n + R - 1) / R;
+  auto load_up = [&](int g, uint4 (&r)[R][NUP][CPT]) {
 #pragma unroll
-    for (int q = 0; q < PC; ++q) {
-      const int c = k * 32 * PC + lane + 32 * q;
-      r[q] = c < nchunks ? ldg_stream(row + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
-    }
-  };
-  float s[V];
+    for (int j = 0; j < R; ++j) {
+      const int i = g * R + j;
+      const int nid = i < n ? ids[i] : -1;
 #pragma unroll
-  for (int v = 0; v < V; ++v) s[v] = 0.f;
-  // biases of this warp's neurons, requested up front: lane l holds neuron
-  // l (and l + 32) of the warp's sequence, fetched by a shuffle when needed
-  float bias_lo = 0.f, bias_hi = 0.f;
-  if (p.b_act) {
-    const int i_lo = warp + lane * kLdgWarps, i_hi = warp + (lane + 32) * kLdgWarps;
-    if (lane < my_n && ids[i_lo] >= 0) bias_lo = p.b_act[ids[i_lo]];
-    if (lane + 32 < my_n && ids[i_hi] >= 0) bias_hi = p.b_act[ids[i_hi]];
-  }
-  auto consume_pass = [&](int pp, const uint4 (&r)[PC]) {
-    const int j = pp / (NUP * ppr), rem = pp % (NUP * ppr);
-    const int m = rem / ppr, k = rem % ppr;
-    const int i = warp + j * kLdgWarps;
+      for (int m = 0; m < NUP; ++m) {
+        const uint8_t* row = (m == 0 ? p.w_act : p.w_up) + (size_t)(nid < 0 ? 0 : nid) * rb;
 #pragma unroll
-    for (int q = 0; q < PC; ++q) {
-      const int c = k * 32 * PC + lane + 32 * q;
-      if (c < nchunks) {
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-          const float dv = dot8<WDT>(r[q], xs + (size_t)b * d + (size_t)c * 8);
-#pragma unroll
-          for (int mm = 0; mm < NUP; ++mm)
-            if (mm == m) s[mm * B + b] += dv;
+        for (int c = 0; c < CPT; ++c) {
+          const int u = t + kLdgThreads * c;
+          r[j][m][c] = (nid >= 0 && u < nchunks) ? ldg_stream_hint(row + (size_t)u * 16, pol)
+                                                 : make_uint4(0, 0, 0, 0);
         }
       }
     }
-    if (rem == NUP * ppr - 1) {  // last pass of neuron i: reduce and store h
-      const float tot = warp_reduce_transposed<V>(s);
-      const int vi = lane >> SH;  // lane (v << SH) holds value v = m*B + b
-      float up = 1.f;
-      if constexpr (ACT == 1) up = __shfl_sync(0xffffffffu, tot, ((vi + B) % V) << SH);
-      const float bi = __shfl_sync(0xffffffffu, j < 32 ? bias_lo : bias_hi, j & 31);
-      if ((lane & ((1 << SH) - 1)) == 0 && vi < B) {
-        float h = fmaxf(tot + bi, 0.f);
-        if constexpr (ACT == 1) h *= up;
-        hs[(size_t)i * B + vi] = ids[i] < 0 ? 0.f : h;
-      }
+  };
+  uint4 ua[R][NUP][CPT], ub[R][NUP][CPT];
+  if (ngroups > 0) load_up(0, ua);
+  // biases of the slice: read only after the first group's barrier
+  for (int i = t; i < n; i += kLdgThreads)
+    lbias[i] = (p.b_act && ids[i] >= 0) ? p.b_act[ids[i]] : 0.f;
+  float xr[B][CPT][8];
 #pragma unroll
-      for (int v = 0; v < V; ++v) s[v] = 0.f;
+  for (int b = 0; b < B; ++b)
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) widen8<WDT>(xq[b][c], xr[b][c]);
+
+  auto consume_up = [&](int g, const uint4 (&r)[R][NUP][CPT]) {
+    float v[VG];
+#pragma unroll
+    for (int j = 0; j < R; ++j)
+#pragma unroll
+      for (int m = 0; m < NUP; ++m)
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          float z = 0.f;
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) z += dot8<WDT>(r[j][m][c], xr[b][c]);
+          v[(j * NUP + m) * B + b] = z;
+        }
+    const float tot = warp_reduce_transposed<VG>(v);
+    const int buf = g & 1;
+    if ((lane & ((1 << SHG) - 1)) == 0) red[buf][warp][lane >> SHG] = tot;
+    __syncthreads();
+    if (t < R * B) {
+      const int j = t / B, b = t % B, i = g * R + j;
+      if (i < n) {
+        float act = 0.f, up = 1.f;
+#pragma unroll
+        for (int w = 0; w < kLdgWarps; ++w) act += red[buf][w][(j * NUP) * B + b];
+        if constexpr (ACT == 1) {
+          up = 0.f;
+#pragma unroll
+          for (int w = 0; w < kLdgWarps; ++w) up += red[buf][w][(j * NUP + 1) * B + b];
+        }
+        const float h = fmaxf(act + lbias[i], 0.f) * up;
+        hs[(size_t)i * B + b] = ids[i] < 0 ? 0.f : h;
+      }
     }
   };
 
-  uint4 ra[PC], rbuf[PC];
-  if (P > 0) load_pass(0, ra);  // in flight while x is staged
-
-  for (int j = t; j < B * d / 8; j += kLdgThreads) {
-    const uint4 v = *reinterpret_cast<const uint4*>(p.x + (size_t)j * 8);
-    widen8<WDT>(v, xs + (size_t)j * 8);
-  }
-  __syncthreads();
-
-  for (int pp = 0; pp < P; pp += 2) {
-    if (pp + 1 < P) load_pass(pp + 1, rbuf);
-    consume_pass(pp, ra);
-    if (pp + 1 < P) {
-      if (pp + 2 < P) load_pass(pp + 2, ra);
-      consume_pass(pp + 1, rbuf);
+  for (int g = 0; g < ngroups; g += 2) {
+    if (g + 1 < ngroups) load_up(g + 1, ub);
+    consume_up(g, ua);
+    if (g + 1 < ngroups) {
+      if (g + 2 < ngroups) load_up(g + 2, ua);
+      consume_up(g + 1, ub);
     }
   }
 
@@ -336,7 +369,7 @@ __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
 #pragma unroll
       for (int c = 0; c < CPT; ++c) {
         const int u = t + kLdgThreads * c;
-        r[j][c] = (i < n && u < nchunks) ? ldg_stream(row + (size_t)u * 16)
+        r[j][c] = (i < n && u < nchunks) ? ldg_stream_hint(row + (size_t)u * 16, pol)
                                          : make_uint4(0, 0, 0, 0);
       }
     }
@@ -419,7 +452,6 @@ __global__ void __launch_bounds__(32 * (NCW + 1), B == 1 ? 2 : 1) k_ffn_tma(FfnP
   constexpr int NUP = ACT == 1 ? 2 : 1;      // dot products per neuron
   constexpr int V = kGroup * NUP * B;        // values reduced per group
   constexpr int SH = 5 - log2c<V>();
-  constexpr int XDT = WDT == 1 ? 1 : 0;      // activation dtype
   constexpr int UE = WDT == 2 ? 32 : 8;      // elements per unit
   const int NS = p.nstages;
 
@@ -430,8 +462,9 @@ __global__ void __launch_bounds__(32 * (NCW + 1), B == 1 ? 2 : 1) k_ffn_tma(FfnP
   float* lbias = reinterpret_cast<float*>(ids + p.list_cap);       // [list_cap]
   float* red = lbias + p.list_cap;                                 // [2][NCW][V]
   float* hs = red + 2 * NCW * V;                                   // [2][kGroup * B]
+  uint32_t* wbuf = reinterpret_cast<uint32_t*>(hs + 2 * kGroup * B); // [2 x F/32]
   uint8_t* stages = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(hs + 2 * kGroup * B) + 127) & ~uintptr_t(127));
+      (reinterpret_cast<uintptr_t>(wbuf + 2 * (p.F / 32)) + 127) & ~uintptr_t(127));
   const uint32_t rb = p.row_bytes;
   const uint32_t stage_bytes = rb * NM;
 
@@ -447,7 +480,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), B == 1 ? 2 : 1) k_ffn_tma(FfnP
   pdl_wait();  // the list (or mask) and x come from earlier kernels
 
   int k0, k1;
-  build_slice<NT>(p, scratch, ids, lbias, k0, k1);
+  build_slice<NT>(p, scratch, wbuf, ids, lbias, k0, k1);
   const int n = k1 - k0;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
