@@ -105,7 +105,7 @@ WsLayout ws_layout(int d, int F, int r, int B) {
   WsLayout w{};
   size_t o = 0;
   w.bar = o;   o += 256;
-  w.a = o;     o += al256((size_t)B * r * 4);
+  w.a = o;     o += al256((size_t)kAReplicas * B * r * 4);
   w.mask = o;  o += al256((size_t)B * (F / 32) * 4);
   w.idx = o;   o += al256((size_t)F * 4);
   w.count = o; o += 256;
@@ -757,7 +757,7 @@ int32_t pi_predict(const pi_predictor* pred, const void* x, int32_t batch, uint3
   if (!aligned16(x) || !aligned16(mask_bits) || (logits && !aligned16(logits)))
     return fail(PI_ERR_INVALID_ARG, "x, mask_bits and logits must be 16-byte aligned");
   const WsLayout w = ws_layout(pred->d_model, pred->d_ff, pred->rank, batch);
-  if (int32_t s = check_ws(workspace, workspace_bytes, w.a + (size_t)batch * pred->rank * 4)) return s;
+  if (int32_t s = check_ws(workspace, workspace_bytes, w.a + (size_t)kAReplicas * batch * pred->rank * 4)) return s;
   float* a = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.a);
   uint32_t* bar = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + w.bar);
   cudaStream_t st = static_cast<cudaStream_t>(stream);

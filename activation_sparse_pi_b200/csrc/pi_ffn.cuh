@@ -674,8 +674,11 @@ __global__ void __launch_bounds__(32 * (NCW + 1), B == 1 ? 2 : 1) k_ffn_tma(FfnP
 // float4 columns with 32 slices each; slice s adds partials g = s, s+32, ...
 // in increasing g, and the 32 slice sums are then added in slice order, so the
 // summation order is fixed and y is reproducible.
-constexpr int kRedCols = 8;
-constexpr int kRedSlices = 32;
+#ifndef PI_RED_COLS
+#define PI_RED_COLS 4
+#endif
+constexpr int kRedCols = PI_RED_COLS;
+constexpr int kRedSlices = 256 / kRedCols;
 
 template <int MODE>
 __global__ void __launch_bounds__(kRedCols * kRedSlices) k_reduce(const float* __restrict__ part,

@@ -376,7 +376,7 @@ struct PredParams {
   const uint16_t* x;       // [B x d] 16-bit input (when x_resid is null)
   const float* x_resid;    // [B x d] fp32 residual stream, or null
   uint16_t* x_out;         // [B x d] rounded layer input (written when x_resid)
-  float* a;                // [B x r] fp32
+  float* a;                // [kAReplicas x B x r] fp32
   const uint8_t* w2;       // [F x r] 16-bit rows
   const float* b2;         // [F]
   uint8_t* mask;           // [B x F/8] bytes: the uint32 mask words, byte-addressed
@@ -393,6 +393,9 @@ constexpr int kPredThreads = 256;
 constexpr int kPredWarps = kPredThreads / 32;
 constexpr int kPredMaxUnits = 64;  // units of 8 rows per CTA
 constexpr int kPredMaxRows1 = 32;  // W1 rows per CTA
+// a is written in several copies and CTA c reads copy c mod kAReplicas, so
+// the grid's reads right after the barrier spread over more L2 lines
+constexpr int kAReplicas = 8;
 
 __host__ __device__ constexpr int pred_p2(int B, int CPL) {
   // layer-2 units in flight per warp: about 96 registers for a and the rows
@@ -535,7 +538,10 @@ __global__ void __launch_bounds__(kPredThreads, 2) k_predict(PredParams p) {
 #pragma unroll
         for (int k = 0; k < kPredWarps; ++k) z += red1[buf][k][t];
         z += bias1[i];
-        p.a[(size_t)b * p.r + c + i * G] = fmaxf(z, 0.f);
+        z = fmaxf(z, 0.f);
+#pragma unroll
+        for (int rep = 0; rep < kAReplicas; ++rep)
+          p.a[((size_t)rep * B + b) * p.r + c + i * G] = z;
       }
     }
   }
@@ -564,7 +570,8 @@ __global__ void __launch_bounds__(kPredThreads, 2) k_predict(PredParams p) {
 #pragma unroll
     for (int k = 0; k < CPL; ++k) {
       const int cc = lane + 32 * k;
-      const float4* src = reinterpret_cast<const float4*>(p.a + (size_t)b * p.r) + 2 * cc;
+      const float4* src =
+          reinterpret_cast<const float4*>(p.a + ((size_t)(c % kAReplicas) * B + b) * p.r) + 2 * cc;
       const float4 lo = cc < nch2 ? __ldcg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
       const float4 hi = cc < nch2 ? __ldcg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
       av[b][k][0] = lo.x; av[b][k][1] = lo.y; av[b][k][2] = lo.z; av[b][k][3] = lo.w;
