@@ -18,8 +18,9 @@ What it computes, and where the pages state it:
 * The neuron-aware operator computes the active neurons' individual row and
   column vectors directly, without converting to a sparse format (unite.ai
   page, section "Neuronenbewusster Operator").
-* Models use ReLU or ReGLU activations (GeekNews page, limitations list);
-  weights may be INT4 Q4_0 (GeekNews page, "Quantization and compatibility").
+* Models use ReLU, ReGLU or Squared-ReLU activations (GeekNews page, summary
+  and limitations list); weights may be INT4 Q4_0 (GeekNews page,
+  "Quantization and compatibility").
 
 The pages give no formulas.  The readings used here are the plain ones:
 
@@ -29,6 +30,8 @@ The pages give no formulas.  The readings used here are the plain ones:
   ascending neuron order, and every token is computed on the whole union;
 * ReLU neuron:  h_i = max(W_up[i] . x + b_up[i], 0);
   ReGLU neuron: h_i = max(W_gate[i] . x + b_gate[i], 0) * (W_up[i] . x);
+  Squared-ReLU neuron: h_i = max(W_up[i] . x + b_up[i], 0)^2 (the pages name
+  the family only; squaring the ReLU output is its definition);
 * output: y = sum over active i of h_i W_down^T[i] (no down bias);
 * stack: pre-norm residual chain, x_l = round16(x_resid / rms(x_resid)),
   x_resid <- x_resid + FFN_l(x_l), where rms is sqrt(mean(x^2) + 1e-6) and
@@ -128,7 +131,7 @@ def round16(x: np.ndarray, dtype: str) -> np.ndarray:
 class OracleLayer:
     d_model: int
     d_ff: int
-    act: str                     # "relu" | "reglu"
+    act: str                     # "relu" | "reglu" | "sqrelu"
     wdtype: str                  # FFN matrices: "f16" | "bf16" | "q4_0"
     pdtype: str                  # predictor matrices: "f16" | "bf16"
     w1: np.ndarray               # stored [r x d]
@@ -189,11 +192,12 @@ def neuron_outputs(layer: OracleLayer, x: np.ndarray, idx: np.ndarray) -> np.nda
     x = np.atleast_2d(np.asarray(x, dtype=np.float64))
     idx = np.asarray(idx, dtype=np.int64)
     up = layer.rows("w_up", idx)
-    if layer.act == "relu":
+    if layer.act in ("relu", "sqrelu"):
         pre = x @ up.T
         if layer.b_up is not None:
             pre = pre + np.asarray(layer.b_up, dtype=np.float64)[idx]
-        return np.maximum(pre, 0.0)
+        r = np.maximum(pre, 0.0)
+        return r if layer.act == "relu" else r * r
     if layer.act == "reglu":
         gate = layer.rows("w_gate", idx)
         g = x @ gate.T
@@ -220,8 +224,9 @@ def dense_ffn(layer: OracleLayer, x: np.ndarray) -> np.ndarray:
 
 
 def true_support(layer: OracleLayer, x: np.ndarray) -> np.ndarray:
-    """[B x F] bool: neurons whose activation is nonzero (ReLU: pre-activation
-    > 0; ReGLU: gate pre-activation > 0 and up projection nonzero)."""
+    """[B x F] bool: neurons whose activation is nonzero (ReLU and Squared-ReLU:
+    pre-activation > 0; ReGLU: gate pre-activation > 0 and up projection
+    nonzero)."""
     return neuron_outputs(layer, x, np.arange(layer.d_ff)) != 0.0
 
 

@@ -53,11 +53,23 @@ def _outputs_reglu_swapped(layer, x, idx):
     return np.maximum(g, 0.0) * (x @ gate.T)
 
 
+def _outputs_sqrelu_unsquared(layer, x, idx):
+    if layer.act != "sqrelu":
+        return _ORIG["neuron_outputs"](layer, x, idx)
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    pre = x @ layer.rows("w_up", idx).T
+    if layer.b_up is not None:
+        pre = pre + np.asarray(layer.b_up)[idx]
+    return np.maximum(pre, 0.0)
+
+
 def _outputs_drop_bias(layer, x, idx):
     x = np.atleast_2d(np.asarray(x, dtype=np.float64))
     up = layer.rows("w_up", idx)
     if layer.act == "relu":
         return np.maximum(x @ up.T, 0.0)
+    if layer.act == "sqrelu":
+        return np.maximum(x @ up.T, 0.0) ** 2
     gate = layer.rows("w_gate", idx)
     return np.maximum(x @ gate.T, 0.0) * (x @ up.T)
 
@@ -113,6 +125,7 @@ MUTANTS = [
     ("masked_ffn", _masked_wrong_row),
     ("neuron_outputs", _outputs_reglu_swapped),
     ("neuron_outputs", _outputs_drop_bias),
+    ("neuron_outputs", _outputs_sqrelu_unsquared),
     ("dequant_q4_0", _dequant_nibbles_swapped),
     ("dequant_q4_0", _dequant_offset7),
     ("union_index", _union_intersection),
@@ -125,6 +138,7 @@ PIN_CASES = [
     (pins.test_predict_and_ffn_brute_force, dict(act="reglu", shape=(48, 16, 6))),
     (pins.test_every_subset_closed_form, dict(act="relu")),
     (pins.test_every_subset_closed_form, dict(act="reglu")),
+    (pins.test_predict_and_ffn_brute_force, dict(act="sqrelu", shape=(16, 8, 4))),
     (pins.test_tie_is_inactive, {}),
     (pins.test_fig8_worked_example, {}),
     (pins.test_union_index_brute_force, {}),

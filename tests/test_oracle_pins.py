@@ -41,6 +41,9 @@ def bf_predict(W1, b1, W2, b2, x, tau):
 def bf_h(act, Wup, Wgate, bup, bgate, x, i):
     if act == "relu":
         return max(bf_dot(Wup[i], x) + (bup[i] if bup is not None else 0.0), 0.0)
+    if act == "sqrelu":
+        r = max(bf_dot(Wup[i], x) + (bup[i] if bup is not None else 0.0), 0.0)
+        return r * r
     g = max(bf_dot(Wgate[i], x) + (bgate[i] if bgate is not None else 0.0), 0.0)
     return g * bf_dot(Wup[i], x)
 
@@ -80,7 +83,7 @@ def tiny_layer(rng, d, F, r, act, tau=0.0, bias=True):
         w1=W1.view(np.uint16), b1=b1, w2=W2.view(np.uint16), b2=b2, threshold=tau,
         w_up=Wup.view(np.uint16), w_gate=None if Wgate is None else Wgate.view(np.uint16),
         w_down_t=Wdt.view(np.uint16),
-        b_up=bact if act == "relu" else None, b_gate=bact if act == "reglu" else None,
+        b_up=bact if act != "reglu" else None, b_gate=bact if act == "reglu" else None,
     )
     lists = dict(
         W1=W1.astype(float).tolist(), W2=W2.astype(float).tolist(),
@@ -88,7 +91,7 @@ def tiny_layer(rng, d, F, r, act, tau=0.0, bias=True):
         Wgate=None if Wgate is None else Wgate.astype(float).tolist(),
         Wdt=Wdt.astype(float).tolist(), b1=b1.astype(float).tolist(),
         b2=b2.astype(float).tolist(),
-        bup=bact.astype(float).tolist() if (bias and act == "relu") else None,
+        bup=bact.astype(float).tolist() if (bias and act != "reglu") else None,
         bgate=bact.astype(float).tolist() if (bias and act == "reglu") else None,
     )
     return L, lists
@@ -101,7 +104,7 @@ def tokens16(rng, B, d):
 # ---------------------------------------------------------------------------
 # masked FFN and predictor against brute force
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("act", ["relu", "reglu"])
+@pytest.mark.parametrize("act", ["relu", "reglu", "sqrelu"])
 @pytest.mark.parametrize("shape", [(16, 8, 4), (48, 16, 6), (64, 12, 8)])
 def test_predict_and_ffn_brute_force(act, shape):
     d, F, r = shape
@@ -126,7 +129,7 @@ def test_predict_and_ffn_brute_force(act, shape):
         np.testing.assert_allclose(yd[b], ybd, rtol=1e-12, atol=1e-12)
 
 
-@pytest.mark.parametrize("act", ["relu", "reglu"])
+@pytest.mark.parametrize("act", ["relu", "reglu", "sqrelu"])
 def test_every_subset_closed_form(act):
     """Every index set I of an F = 8 layer: y(I) = y_dense - sum over
     support-minus-I of h_i W_down^T[i]."""
@@ -152,7 +155,7 @@ def test_every_subset_closed_form(act):
             np.testing.assert_allclose(got, expect, rtol=1e-9, atol=1e-11)
 
 
-@pytest.mark.parametrize("act", ["relu", "reglu"])
+@pytest.mark.parametrize("act", ["relu", "reglu", "sqrelu"])
 def test_superset_of_support_equals_dense(act):
     rng = np.random.default_rng(7)
     L, _ = tiny_layer(rng, 32, 16, 4, act)
