@@ -12,6 +12,7 @@ from .binding import (  # noqa: F401
     PI_Q4_0,
     PI_REGLU,
     PI_RELU,
+    PI_SQRELU,
     PiError,
     PiLayer,
     PiPredictor,

@@ -15,9 +15,9 @@ LIB_PATH = os.path.join(HERE, "libpi.so")
 PI_OK, PI_ERR_INVALID_ARG, PI_ERR_UNSUPPORTED, PI_ERR_WORKSPACE, PI_ERR_CUDA = range(5)
 PI_STATIC_SCRATCH_BYTES = 16 << 20  # fixed scratch of pi_sparse_ffn_static
 PI_F16, PI_BF16, PI_Q4_0 = 0, 1, 2
-PI_RELU, PI_REGLU = 0, 1
+PI_RELU, PI_REGLU, PI_SQRELU = 0, 1, 2
 DTYPES = {"f16": PI_F16, "bf16": PI_BF16, "q4_0": PI_Q4_0}
-ACTS = {"relu": PI_RELU, "reglu": PI_REGLU}
+ACTS = {"relu": PI_RELU, "reglu": PI_REGLU, "sqrelu": PI_SQRELU}
 
 EXPORTS = (
     "pi_status_string", "pi_last_error", "pi_device_error", "pi_launch_count", "pi_workspace_size",

@@ -189,8 +189,8 @@ int32_t validate_layer(const pi_layer* L) {
     return fail(PI_ERR_INVALID_ARG, "layer and predictor disagree on d_model/d_ff");
   if (!check_act_dtype(L->adtype) || L->adtype != L->pred.dtype)
     return fail(PI_ERR_UNSUPPORTED, "adtype must be PI_F16/PI_BF16 and equal the predictor dtype");
-  if (L->act != PI_RELU && L->act != PI_REGLU)
-    return fail(PI_ERR_UNSUPPORTED, "act must be PI_RELU or PI_REGLU");
+  if (L->act != PI_RELU && L->act != PI_REGLU && L->act != PI_SQRELU)
+    return fail(PI_ERR_UNSUPPORTED, "act must be PI_RELU, PI_REGLU or PI_SQRELU");
   if (L->wdtype == PI_F16 || L->wdtype == PI_BF16) {
     if (L->wdtype != L->adtype)
       return fail(PI_ERR_UNSUPPORTED, "16-bit weights must have the activation dtype");
@@ -204,7 +204,7 @@ int32_t validate_layer(const pi_layer* L) {
   if (!L->w_up || !L->w_down_t) return fail(PI_ERR_INVALID_ARG, "w_up and w_down_t are required");
   if ((L->act == PI_REGLU) != (L->w_gate != nullptr))
     return fail(PI_ERR_INVALID_ARG, "w_gate must be given exactly for ReGLU");
-  if (L->act == PI_RELU && L->b_gate)
+  if (L->act != PI_REGLU && L->b_gate)
     return fail(PI_ERR_INVALID_ARG, "b_gate is only meaningful for ReGLU");
   if (L->act == PI_REGLU && L->b_up)
     return fail(PI_ERR_INVALID_ARG, "ReGLU has no up-projection bias (use b_gate)");
@@ -637,6 +637,14 @@ cudaError_t launch_up_generic(const pi_layer* L, int B, const uint16_t* x, const
   return launch(k_rows<kModeUp, WDT, ACT, 64>, dim3(blocks), dim3(256), 0, st, p);
 }
 
+template <int WDT>
+cudaError_t up_generic_act(const pi_layer* L, int B, const uint16_t* x, const int32_t* idx,
+                           const int32_t* count, float* h, cudaStream_t st) {
+  if (L->act == PI_REGLU) return launch_up_generic<WDT, 1>(L, B, x, idx, count, h, st);
+  if (L->act == PI_SQRELU) return launch_up_generic<WDT, 2>(L, B, x, idx, count, h, st);
+  return launch_up_generic<WDT, 0>(L, B, x, idx, count, h, st);
+}
+
 // Records a caller's timing event on the stream; under stream capture it
 // becomes an external event-record node, so every graph launch records it.
 cudaError_t record_event(void* ev, cudaStream_t st) {
@@ -663,9 +671,21 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     cudaError_t e = cudaErrorInvalidValue;
     const int act = L->act;
     switch (L->wdtype) {
-      case PI_F16: e = act ? ffn_ldg<0, 1>(L, B, x, src, part, st) : ffn_ldg<0, 0>(L, B, x, src, part, st); break;
-      case PI_BF16: e = act ? ffn_ldg<1, 1>(L, B, x, src, part, st) : ffn_ldg<1, 0>(L, B, x, src, part, st); break;
-      case PI_Q4_0: e = act ? ffn_tma<1>(L, B, x, src, part, st) : ffn_tma<0>(L, B, x, src, part, st); break;
+      case PI_F16:
+        e = act == PI_REGLU ? ffn_ldg<0, 1>(L, B, x, src, part, st)
+          : act == PI_SQRELU ? ffn_ldg<0, 2>(L, B, x, src, part, st)
+                             : ffn_ldg<0, 0>(L, B, x, src, part, st);
+        break;
+      case PI_BF16:
+        e = act == PI_REGLU ? ffn_ldg<1, 1>(L, B, x, src, part, st)
+          : act == PI_SQRELU ? ffn_ldg<1, 2>(L, B, x, src, part, st)
+                             : ffn_ldg<1, 0>(L, B, x, src, part, st);
+        break;
+      case PI_Q4_0:
+        e = act == PI_REGLU ? ffn_tma<1>(L, B, x, src, part, st)
+          : act == PI_SQRELU ? ffn_tma<2>(L, B, x, src, part, st)
+                             : ffn_tma<0>(L, B, x, src, part, st);
+        break;
     }
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "fused FFN launch failed: %s", cudaGetErrorString(e));
     G = ffn_grid(B);
@@ -675,9 +695,9 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     cudaError_t e = cudaErrorInvalidValue;
     const int act = L->act;
     switch (L->wdtype) {
-      case PI_F16: e = act ? launch_up_generic<0, 1>(L, B, x, src.idx, src.count, h, st) : launch_up_generic<0, 0>(L, B, x, src.idx, src.count, h, st); break;
-      case PI_BF16: e = act ? launch_up_generic<1, 1>(L, B, x, src.idx, src.count, h, st) : launch_up_generic<1, 0>(L, B, x, src.idx, src.count, h, st); break;
-      case PI_Q4_0: e = act ? launch_up_generic<2, 1>(L, B, x, src.idx, src.count, h, st) : launch_up_generic<2, 0>(L, B, x, src.idx, src.count, h, st); break;
+      case PI_F16: e = up_generic_act<0>(L, B, x, src.idx, src.count, h, st); break;
+      case PI_BF16: e = up_generic_act<1>(L, B, x, src.idx, src.count, h, st); break;
+      case PI_Q4_0: e = up_generic_act<2>(L, B, x, src.idx, src.count, h, st); break;
     }
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "batched up launch failed: %s", cudaGetErrorString(e));
     DownParams dp{};

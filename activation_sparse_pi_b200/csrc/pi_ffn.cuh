@@ -238,8 +238,8 @@ constexpr int kLdgWarps = kLdgThreads / 32;
 constexpr int kUpRegs = PI_UP_REGS;      // up phase: 16-byte loads per thread per buffer
 constexpr int kDownRegs = PI_DOWN_REGS;  // down phase: 16-byte loads per thread per buffer
 
-// WDT: 0 fp16, 1 bf16 (activations of the same type).  ACT: 0 ReLU, 1 ReGLU.
-// CPT: column chunks per thread.  CPS: CTAs per SM.
+// WDT: 0 fp16, 1 bf16 (activations of the same type).  ACT: 0 ReLU, 1 ReGLU,
+// 2 Squared-ReLU.  CPT: column chunks per thread.  CPS: CTAs per SM.
 template <int WDT, int ACT, int B, int CPT, int CPS>
 __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -344,7 +344,8 @@ __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
 #pragma unroll
           for (int w = 0; w < kLdgWarps; ++w) up += red[buf][w][(j * NUP + 1) * B + b];
         }
-        const float h = fmaxf(act + lbias[i], 0.f) * up;
+        const float r = fmaxf(act + lbias[i], 0.f);
+        const float h = ACT == 2 ? r * r : r * up;
         hs[(size_t)i * B + b] = ids[i] < 0 ? 0.f : h;
       }
     }
@@ -604,6 +605,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), B == 1 ? 2 : 1) k_ffn_tma(FfnP
         const int i = g + q;
         h = fmaxf(sa + lbias[i], 0.f);
         if constexpr (ACT == 1) h *= su;
+        if constexpr (ACT == 2) h *= h;
         if (ids[i] < 0) h = 0.f;
       }
       hs[buf * kGroup * B + ct] = h;

@@ -177,6 +177,7 @@ __global__ void __launch_bounds__(256) k_rows(RowsParams p) {
         } else {
           float h = fmaxf(tot[0] + (valid ? bias : 0.f), 0.f);
           if constexpr (ACT == 1) h *= tot[NUP - 1];
+          if constexpr (ACT == 2) h *= h;
           if (!valid) h = 0.f;
           p.out[(size_t)row * B + b] = h;
         }

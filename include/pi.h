@@ -58,7 +58,11 @@ typedef enum {
 } pi_status;
 
 typedef enum { PI_F16 = 0, PI_BF16 = 1, PI_Q4_0 = 2 } pi_dtype;
-typedef enum { PI_RELU = 0, PI_REGLU = 1 } pi_act;
+/* Neuron activation (GeekNews page, summary and limitations list: ReLU,
+ * ReGLU and Squared-ReLU models are supported).  ReLU: h = max(u, 0) with
+ * u = W_up[i].x + b_up[i]; ReGLU: h = max(g, 0) * (W_up[i].x) with
+ * g = W_gate[i].x + b_gate[i]; Squared-ReLU: h = max(u, 0)^2. */
+typedef enum { PI_RELU = 0, PI_REGLU = 1, PI_SQRELU = 2 } pi_act;
 
 /*
  * Activation predictor of one layer (unite.ai page, "Adaptive

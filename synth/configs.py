@@ -17,7 +17,7 @@ class Config:
     n_layers: int
     d_model: int
     d_ff: int
-    act: str              # "relu" or "reglu"
+    act: str              # "relu", "reglu" or "sqrelu"
     wdtype: str           # "f16", "bf16" or "q4_0" (FFN matrices)
     adtype: str           # 16-bit activation / predictor dtype: "f16" or "bf16"
     sigma_w: float        # std of the FFN weights
@@ -52,6 +52,10 @@ CONFIGS = {
                n_tokens=128, prompt_tokens=64),
         Config(4, "llama2-70b-q4", 80, 8192, 28672, "reglu", "q4_0", "f16", 0.015, 1.1, 0.10,
                1536, batches=(1, 8, 32), n_tokens=128),
+        # the OPT-6.7B shapes with Squared-ReLU neurons (GeekNews page, limitations
+        # list: ReLU, ReGLU and Squared-ReLU models)
+        Config(5, "opt-6.7b-sqrelu", 32, 4096, 16384, "sqrelu", "f16", "f16", 0.02, 1.1, 0.20,
+               1024, n_tokens=128),
     ]
 }
 

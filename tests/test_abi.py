@@ -106,6 +106,9 @@ def test_predict_rejects_batch_and_workspace(lib):
     (dict(w_gate=FAKE), pi.binding.PI_ERR_INVALID_ARG),              # gate for ReLU
     (dict(wdtype="bf16"), pi.binding.PI_ERR_UNSUPPORTED),            # weights != activations
     (dict(wdtype="q4_0", d_model=512), 0),                           # allowed (d % 256 == 0)
+    (dict(act="sqrelu"), 0),                                         # Squared-ReLU: like ReLU
+    (dict(act="sqrelu", w_gate=FAKE), pi.binding.PI_ERR_INVALID_ARG),  # no gate
+    (dict(act="sqrelu", b_gate=FAKE), pi.binding.PI_ERR_INVALID_ARG),
     (dict(wdtype="q4_0", d_model=480, pred=_pred(d_model=480)), pi.binding.PI_ERR_UNSUPPORTED),
     (dict(adtype="bf16"), pi.binding.PI_ERR_UNSUPPORTED),            # != predictor dtype
     (dict(d_ff=1024), pi.binding.PI_ERR_INVALID_ARG),                # != predictor d_ff

@@ -30,6 +30,9 @@ SMALL = {
         Config(13, "t-q4-reglu", 3, 512, 1536, "reglu", "q4_0", "f16", 0.015, 1.1, 0.1, 128),
         Config(14, "t-q4-relu", 2, 768, 2048, "relu", "q4_0", "f16", 0.015, 1.1, 0.1, 256),
         Config(15, "t-relu-f16-8192", 2, 8192, 1024, "relu", "f16", "f16", 0.015, 1.0, 0.08, 512),
+        Config(16, "t-sqrelu-f16", 3, 1024, 4096, "sqrelu", "f16", "f16", 0.02, 1.1, 0.15, 256),
+        Config(17, "t-sqrelu-bf16-2560", 2, 2560, 2048, "sqrelu", "bf16", "bf16", 0.02, 1.1, 0.15, 256),
+        Config(18, "t-q4-sqrelu", 2, 512, 2048, "sqrelu", "q4_0", "f16", 0.015, 1.1, 0.1, 128),
     ]
 }
 BATCHES = [1, 2, 4, 8, 32]
@@ -307,7 +310,8 @@ def test_stack_deterministic():
 # ------------------------------------------------- full sizes (sampled)
 FULL_LAYER_CASES = [("opt-6.7b", 1), ("opt-6.7b", 4), ("relu-llama2-13b", 1),
                     ("relu-llama2-13b", 8), ("falcon-40b", 1), ("falcon-40b", 64),
-                    ("llama2-70b-q4", 1), ("llama2-70b-q4", 8), ("llama2-70b-q4", 32)]
+                    ("llama2-70b-q4", 1), ("llama2-70b-q4", 8), ("llama2-70b-q4", 32),
+                    ("opt-6.7b-sqrelu", 1)]
 
 
 @pytest.mark.slow
