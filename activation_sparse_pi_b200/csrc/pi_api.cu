@@ -482,7 +482,6 @@ size_t ffn_row_bytes(const pi_layer* L) {
   return L->wdtype == PI_Q4_0 ? (size_t)L->d_model / 32 * 18 : (size_t)L->d_model * 2;
 }
 
-int ffn_nm(const pi_layer* L) { return L->act == PI_REGLU ? 3 : 2; }
 
 int ffn_list_cap(const pi_layer* L, int B) {
   return (L->d_ff + ffn_grid(B) - 1) / ffn_grid(B) + 1;
@@ -500,31 +499,12 @@ size_t ldg_smem(const pi_layer* L, int B) {
   return 256 + (size_t)ffn_list_cap(L, B) * (8 + 4 * B) + (size_t)L->d_ff / 4 + 16;
 }
 
-// Q4_0 weights (k_ffn_tma): 8 consumer warps, kTmaLanes producer lanes
-constexpr int kTmaNcw = 8;
-constexpr int kTmaLanes = 2;
-
-size_t tma_fixed_smem(const pi_layer* L, int B) {
-  const int V = kGroup * (L->act == PI_REGLU ? 2 : 1) * B;
-  return 1024 + (size_t)ffn_list_cap(L, B) * 8 + (size_t)2 * kTmaNcw * V * 4 +
-         (size_t)2 * kGroup * B * 4 + (size_t)L->d_ff / 4 + 128;
-}
-
-int tma_nstages(const pi_layer* L, int B) {
-  const size_t stage = ffn_row_bytes(L) * ffn_nm(L);
-  const size_t fixed = tma_fixed_smem(L, B);
-  const size_t budget = kSmemFfn / ffn_cps(B);
-  if (fixed >= budget) return 0;
-  int ns = (int)std::min<size_t>(32, (budget - fixed) / stage);
-  return ns - ns % kTmaLanes;  // each producer lane owns whole stages
-}
-
 bool ffn_fused_ok(const pi_layer* L, int B) {
   if (!(B == 1 || B == 2 || B == 4)) return false;
   if (L->wdtype == PI_Q4_0) {
-    // one 32-element block per consumer thread
-    if (L->d_model / 32 > 32 * kTmaNcw || B > 2) return false;
-    return tma_nstages(L, B) >= kGroup;
+    // one 32-element block per thread (d <= 8192)
+    if (L->d_model / 32 > kQ4Threads || B > 2) return false;
+    return ldg_smem(L, B) <= kSmemFfn / ffn_cps(B);
   }
   const int c = ldg_cpt(L->d_model);
   if (c == 0 || B * c > 8) return false;
@@ -598,21 +578,15 @@ cudaError_t ffn_ldg(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& s
   return ffn_ldg_cpt<WDT, ACT, 4>(L, x, src, part, st);
 }
 
-template <int ACT, int B>
-cudaError_t launch_ffn_tma(const pi_layer* L, const uint16_t* x, const FfnSrc& src, float* part,
-                           cudaStream_t st) {
-  FfnParams p = ffn_params(L, B, x, src, part);
-  p.nstages = tma_nstages(L, B);
-  const size_t smem = tma_fixed_smem(L, B) + (size_t)p.nstages * p.row_bytes * ffn_nm(L);
-  return launch(k_ffn_tma<2, ACT, B, 1, kTmaNcw, kTmaLanes>, dim3(ffn_grid(B)),
-                dim3(32 * (kTmaNcw + 1)), smem, st, p);
-}
-
+// Q4_0 weights: k_ffn_q4, block t of every row on thread t
 template <int ACT>
-cudaError_t ffn_tma(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, float* part,
-                    cudaStream_t st) {
-  if (B == 1) return launch_ffn_tma<ACT, 1>(L, x, src, part, st);
-  if (B == 2) return launch_ffn_tma<ACT, 2>(L, x, src, part, st);
+cudaError_t ffn_q4(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, float* part,
+                   cudaStream_t st) {
+  const FfnParams p = ffn_params(L, B, x, src, part);
+  if (B == 1)
+    return launch(k_ffn_q4<ACT, 1>, dim3(ffn_grid(1)), dim3(kQ4Threads), ldg_smem(L, 1), st, p);
+  if (B == 2)
+    return launch(k_ffn_q4<ACT, 2>, dim3(ffn_grid(2)), dim3(kQ4Threads), ldg_smem(L, 2), st, p);
   return cudaErrorInvalidValue;
 }
 
@@ -682,9 +656,9 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
                              : ffn_ldg<1, 0>(L, B, x, src, part, st);
         break;
       case PI_Q4_0:
-        e = act == PI_REGLU ? ffn_tma<1>(L, B, x, src, part, st)
-          : act == PI_SQRELU ? ffn_tma<2>(L, B, x, src, part, st)
-                             : ffn_tma<0>(L, B, x, src, part, st);
+        e = act == PI_REGLU ? ffn_q4<1>(L, B, x, src, part, st)
+          : act == PI_SQRELU ? ffn_q4<2>(L, B, x, src, part, st)
+                             : ffn_q4<0>(L, B, x, src, part, st);
         break;
     }
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "fused FFN launch failed: %s", cudaGetErrorString(e));
@@ -693,7 +667,6 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     if (src.mask) return fail(PI_ERR_UNSUPPORTED, "mask-driven FFN needs the fused kernel");
     float* h = reinterpret_cast<float*>(ws + w.h);
     cudaError_t e = cudaErrorInvalidValue;
-    const int act = L->act;
     switch (L->wdtype) {
       case PI_F16: e = up_generic_act<0>(L, B, x, src.idx, src.count, h, st); break;
       case PI_BF16: e = up_generic_act<1>(L, B, x, src.idx, src.count, h, st); break;

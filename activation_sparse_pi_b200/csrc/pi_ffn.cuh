@@ -97,7 +97,6 @@ struct FfnParams {
   float* part;             // [gridDim.x x B x d]
   int d, F;
   uint32_t row_bytes;
-  int nstages;             // TMA kernel: ring stages
   int list_cap;
   // weights the next kernels will read (the next layer's predictor), asked
   // of the L2 while this kernel's prologue leaves DRAM idle; null for none
@@ -434,240 +433,280 @@ __global__ void __launch_bounds__(kLdgThreads, CPS) k_ffn_ldg(FfnParams p) {
     }
 }
 
-// ------------------------------------------------ gathered FFN, Q4_0 (TMA)
-// Q4_0 rows (18-byte blocks) are staged whole in shared memory by 1-D bulk
-// copies.  A stage holds one neuron: its activation row (W_up for ReLU, W_gate
-// for ReGLU), its W_up row (ReGLU only) and its W_down^T row.  The consumer
-// warps compute h for a group of kGroup neurons (block-wide dot products: x
-// stays in registers), then add h * W_down^T[n] into fp32 accumulators held
-// in registers for the whole slice.
-constexpr int kGroup = 4;
+// ------------------------------------------------ gathered FFN, Q4_0 (LDG)
+// Q4_0 rows (d/32 blocks of 18 bytes: fp16 scale, then 16 bytes whose byte j
+// holds element j in its low nibble and element j+16 in its high nibble) are
+// streamed through registers like the 16-bit rows.  Thread t owns block t of
+// every row: its 32 elements of x (fp32, in registers) in the up phase and its
+// 32 columns of y in the down phase.  The 32 blocks of warp w form one
+// 16-byte aligned 576-byte span (36 chunks), which the warp loads with
+// 128-bit loads and passes through a 576-byte shared-memory slot so that each
+// lane reads back its own 18 bytes.  Each nibble q becomes the exact float
+// f = 1 + q/16 with one byte permute (exponent byte 0x3F, mantissa byte
+// 0x80 | 8q, prepared four at a time), so a block's dot product is
+//   scale * sum_e (q_e - 8) x_e = scale * (16 sum_e f_e x_e - 24 sum_e x_e)
+// and the down phase adds (16 h scale) f_e per column and -24 h scale once.
+#ifndef PI_Q4_SPANS
+#define PI_Q4_SPANS 4
+#endif
+constexpr int kQ4Threads = 256;
+constexpr int kQ4Warps = kQ4Threads / 32;
+constexpr int kQ4Spans = PI_Q4_SPANS;  // rows in flight per thread per buffer
+constexpr int kQ4SpanBytes = 576;      // 32 blocks x 18 bytes
 
-template <int WDT, int ACT, int B, int CPT, int NCW, int PL>
-__global__ void __launch_bounds__(32 * (NCW + 1), B == 1 ? 2 : 1) k_ffn_tma(FfnParams p) {
-  static_assert(WDT == 2, "the bulk-copy kernel serves Q4_0 weights");
+// This lane's block out of its warp's span in shared memory (144 words).
+__device__ __forceinline__ void q4_lane_block(const uint32_t* span, int lane, uint32_t& sc,
+                                              uint32_t (&q)[4]) {
+  const int w0 = (9 * lane) >> 1;  // word holding byte 18 * lane
+  uint32_t w[5];
+#pragma unroll
+  for (int k = 0; k < 5; ++k) w[k] = span[w0 + k];
+  const bool odd = lane & 1;  // odd lanes start 2 bytes into the word
+  sc = odd ? (w[0] >> 16) : (w[0] & 0xffffu);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) q[k] = odd ? w[k + 1] : __funnelshift_r(w[k], w[k + 1], 16);
+}
+
+// The four low (hi = false) or high nibbles of w, each as the byte 0x80 | 8q.
+__device__ __forceinline__ uint32_t nib_bytes(uint32_t w, bool hi) {
+  return ((hi ? (w >> 1) : (w << 3)) & 0x78787878u) | 0x80808080u;
+}
+// 1 + q/16 for the nibble in byte i of v (from nib_bytes): bits 0x3F800000 | q << 19.
+__device__ __forceinline__ float nib16(uint32_t v, int i) {
+  return __uint_as_float(__byte_perm(v, 0x3F000000u, 0x7044u | ((uint32_t)i << 8)));
+}
+
+template <int ACT, int B>
+__global__ void __launch_bounds__(kQ4Threads, B == 1 ? 2 : 1) k_ffn_q4(FfnParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int NT = 32 * (NCW + 1);
-  constexpr int NCT = 32 * NCW;              // consumer threads
-  constexpr int NM = ACT == 1 ? 3 : 2;       // matrices per stage
-  constexpr int NUP = ACT == 1 ? 2 : 1;      // dot products per neuron
-  constexpr int V = kGroup * NUP * B;        // values reduced per group
-  constexpr int SH = 5 - log2c<V>();
-  constexpr int UE = WDT == 2 ? 32 : 8;      // elements per unit
-  const int NS = p.nstages;
+  constexpr int NUP = ACT == 1 ? 2 : 1;                 // up-phase rows per neuron
+  constexpr int R = kQ4Spans / NUP > 0 ? kQ4Spans / NUP : 1;  // neurons per up group
+  constexpr int VG = R * NUP * B;
+  constexpr int SHG = 5 - log2c<VG>();
+  static_assert(VG <= 32 && (VG & (VG - 1)) == 0, "a group's dot products fit one warp reduction");
+  constexpr int DH = kQ4Spans;                          // down: neurons per buffer
+  int* scratch = reinterpret_cast<int*>(smem);
+  int* ids = reinterpret_cast<int*>(smem + 256);
+  float* lbias = reinterpret_cast<float*>(ids + p.list_cap);
+  float* hs = lbias + p.list_cap;
+  uint32_t* wbuf = reinterpret_cast<uint32_t*>(hs + (size_t)p.list_cap * B);
+  __shared__ __align__(16) uint32_t spans[kQ4Warps][kQ4SpanBytes / 4];
+  __shared__ float red[2][kQ4Warps][VG];
 
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* empty = full + NS;
-  int* scratch = reinterpret_cast<int*>(smem + 512);              // 64 ints
-  int* ids = reinterpret_cast<int*>(smem + 1024);                  // [list_cap]
-  float* lbias = reinterpret_cast<float*>(ids + p.list_cap);       // [list_cap]
-  float* red = lbias + p.list_cap;                                 // [2][NCW][V]
-  float* hs = red + 2 * NCW * V;                                   // [2][kGroup * B]
-  uint32_t* wbuf = reinterpret_cast<uint32_t*>(hs + 2 * kGroup * B); // [2 x F/32]
-  uint8_t* stages = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(wbuf + 2 * (p.F / 32)) + 127) & ~uintptr_t(127));
-  const uint32_t rb = p.row_bytes;
-  const uint32_t stage_bytes = rb * NM;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], NCW);
-    }
-    fence_mbar_init();
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int d = p.d, nb = d / 32;
+  const size_t rb = (size_t)nb * 18;
+  const bool mine = t < nb;                              // this thread owns block t
+  const int nv = min(32, max(0, nb - 32 * warp));        // blocks in this warp's span
+  const int cnt = nv * 9 / 8;                            // 16-byte chunks in the span
+  const uint64_t pol = policy_evict_first();
+  if (t == 0) {
+    prefetch_l2_share(p.pf_base[0], p.pf_bytes[0], blockIdx.x, gridDim.x);
+    prefetch_l2_share(p.pf_base[1], p.pf_bytes[1], blockIdx.x, gridDim.x);
   }
-  __syncthreads();
+
   pdl_trigger();
   pdl_wait();  // the list (or mask) and x come from earlier kernels
-
+  uint4 xq[B][4];
+#pragma unroll
+  for (int b = 0; b < B; ++b)
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      xq[b][k] = mine ? reinterpret_cast<const uint4*>(p.x + (size_t)b * d + (size_t)t * 32)[k]
+                      : make_uint4(0, 0, 0, 0);
   int k0, k1;
-  build_slice<NT>(p, scratch, wbuf, ids, lbias, k0, k1);
+  build_slice<kQ4Threads, false>(p, scratch, wbuf, ids, lbias, k0, k1);
   const int n = k1 - k0;
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp == 0) {
-    // ---------------------------------------------------------- producer
-    if (lane < PL) {
-      const uint64_t pol = policy_evict_first();
-      for (int i = lane; i < n; i += PL) {
-        const int s = i % NS;
-        if (i >= NS && !mbar_wait_sleep(&empty[s], ((i / NS) - 1) & 1)) break;
-        const int nid = ids[i] < 0 ? 0 : ids[i];
-        mbar_arrive_expect_tx(&full[s], stage_bytes);
-        uint8_t* st = stages + (size_t)s * stage_bytes;
-        const size_t off = (size_t)nid * rb;
-        bulk_g2s_hint(st, p.w_act + off, rb, &full[s], pol);
-        if constexpr (ACT == 1) bulk_g2s_hint(st + rb, p.w_up + off, rb, &full[s], pol);
-        bulk_g2s_hint(st + (NM - 1) * rb, p.w_dn + off, rb, &full[s], pol);
-      }
-      // drain this lane's last copies before the CTA can exit
-      for (int i = lane; i < n; i += PL)
-        if (i >= n - NS) mbar_wait_sleep(&full[i % NS], (i / NS) & 1);
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------ consumers
-  const int ct = threadIdx.x - 32;
-  const int cw = warp - 1;
-  const int nunits = p.d / UE;
-
-  constexpr int XW = WDT == 2 ? 32 : 4;  // Q4: 32 fp32 values; 16-bit: 4 packed words
-  uint32_t xr[B][CPT][XW];
-#pragma unroll
-  for (int b = 0; b < B; ++b)
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) {
-      const int u = ct + NCT * c;
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        xr[b][c][e] = (u < nunits) ? __float_as_uint(__half2float(__ushort_as_half(
-                                         p.x[(size_t)b * p.d + u * 32 + e])))
-                                   : 0u;
-    }
-
-  float acc[B][CPT][UE];
-#pragma unroll
-  for (int b = 0; b < B; ++b)
-#pragma unroll
-    for (int c = 0; c < CPT; ++c)
-#pragma unroll
-      for (int e = 0; e < UE; ++e) acc[b][c][e] = 0.f;
-
-  // Every consumer takes part in every group's barriers, so a timed-out wait
-  // only stops this thread's arithmetic, never its barrier arrivals.
-  bool ok = true;
-  int grp = 0;
-  for (int g = 0; g < n; g += kGroup, ++grp) {
-    const int ng = min(kGroup, n - g);
-    const int buf = grp & 1;
-#pragma unroll
-    for (int q = 0; q < kGroup; ++q) {
-      const int i = g + q;
-      if (q < ng && ok && !mbar_wait_sleep(&full[i % NS], (i / NS) & 1)) ok = false;
-    }
-    // partial dot products of this thread's units
-    float v[V];
-#pragma unroll
-    for (int t = 0; t < V; ++t) v[t] = 0.f;
-    if (ok) {
-#pragma unroll
-      for (int q = 0; q < kGroup; ++q) {
-        if (q < ng) {
-          const uint8_t* st = stages + (size_t)((g + q) % NS) * stage_bytes;
-#pragma unroll
-          for (int m = 0; m < NUP; ++m) {
-            const uint8_t* row = st + m * rb;
-#pragma unroll
-            for (int c = 0; c < CPT; ++c) {
-              const int u = ct + NCT * c;
-              if (u < nunits) {
-                if constexpr (WDT == 2) {
-                  const uint8_t* blk = row + (size_t)u * 18;
-                  const uint16_t* h16 = reinterpret_cast<const uint16_t*>(blk);
-                  const float sc = __half2float(__ushort_as_half(h16[0]));
-                  uint32_t qb[4];
-#pragma unroll
-                  for (int e = 0; e < 4; ++e)
-                    qb[e] = (uint32_t)h16[1 + 2 * e] | ((uint32_t)h16[2 + 2 * e] << 16);
-#pragma unroll
-                  for (int b = 0; b < B; ++b) {
-                    float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                      const uint32_t byte = (qb[e >> 2] >> ((e & 3) * 8)) & 0xffu;
-                      s0 = fmaf(q4_val(byte & 15u), __uint_as_float(xr[b][c][e]), s0);
-                      s1 = fmaf(q4_val(byte >> 4), __uint_as_float(xr[b][c][e + 16]), s1);
-                    }
-                    v[(q * NUP + m) * B + b] += (s0 + s1) * sc;
-                  }
-                }
-              }
-            }
-          }
-        }
-      }
-    }
-    // block reduction: warp transposed reduce, then across warps
-    const float tot = warp_reduce_transposed<V>(v);
-    if ((lane & ((1 << SH) - 1)) == 0) red[(buf * NCW + cw) * V + (lane >> SH)] = tot;
-    named_bar_sync(1, NCT);
-    if (ct < kGroup * B) {
-      const int q = ct / B, b = ct % B;
-      float h = 0.f;
-      if (q < ng && ok) {
-        float sa = 0.f, su = 0.f;
-#pragma unroll
-        for (int w = 0; w < NCW; ++w) {
-          sa += red[(buf * NCW + w) * V + (q * NUP + 0) * B + b];
-          if constexpr (ACT == 1) su += red[(buf * NCW + w) * V + (q * NUP + 1) * B + b];
-        }
-        const int i = g + q;
-        h = fmaxf(sa + lbias[i], 0.f);
-        if constexpr (ACT == 1) h *= su;
-        if constexpr (ACT == 2) h *= h;
-        if (ids[i] < 0) h = 0.f;
-      }
-      hs[buf * kGroup * B + ct] = h;
-    }
-    named_bar_sync(1, NCT);
-    // down projection: acc += h * W_down^T[n]
-    if (ok) {
-#pragma unroll
-      for (int q = 0; q < kGroup; ++q) {
-        if (q < ng) {
-          const uint8_t* row = stages + (size_t)((g + q) % NS) * stage_bytes + (NM - 1) * rb;
-          float hq[B];
-#pragma unroll
-          for (int b = 0; b < B; ++b) hq[b] = hs[buf * kGroup * B + q * B + b];
-#pragma unroll
-          for (int c = 0; c < CPT; ++c) {
-            const int u = ct + NCT * c;
-            if (u < nunits) {
-              if constexpr (WDT == 2) {
-                const uint8_t* blk = row + (size_t)u * 18;
-                const uint16_t* h16 = reinterpret_cast<const uint16_t*>(blk);
-                const float sc = __half2float(__ushort_as_half(h16[0]));
-                uint32_t qb[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  qb[e] = (uint32_t)h16[1 + 2 * e] | ((uint32_t)h16[2 + 2 * e] << 16);
-#pragma unroll
-                for (int b = 0; b < B; ++b) {
-                  const float hsc = hq[b] * sc;
-#pragma unroll
-                  for (int e = 0; e < 16; ++e) {
-                    const uint32_t byte = (qb[e >> 2] >> ((e & 3) * 8)) & 0xffu;
-                    acc[b][c][e] = fmaf(hsc, q4_val(byte & 15u), acc[b][c][e]);
-                    acc[b][c][e + 16] = fmaf(hsc, q4_val(byte >> 4), acc[b][c][e + 16]);
-                  }
-                }
-              }
-            }
-          }
-        }
-      }
-    }
+  struct Span { uint4 m, e; };
+  auto load_span = [&](const uint8_t* row, Span& sp) {
+    const uint4* src = reinterpret_cast<const uint4*>(row + (size_t)warp * kQ4SpanBytes);
+    sp.m = lane < cnt ? ldg_stream_hint(src + lane, pol) : make_uint4(0, 0, 0, 0);
+    sp.e = lane + 32 < cnt ? ldg_stream_hint(src + 32 + lane, pol) : make_uint4(0, 0, 0, 0);
+  };
+  // pass a span through the warp's slot; returns this lane's scale and nibbles
+  auto open_span = [&](const Span& sp, float& scale, uint32_t (&q)[4]) {
+    uint4* slot = reinterpret_cast<uint4*>(spans[warp]);
     __syncwarp();
-    if (lane == 0)
-      for (int q = 0; q < ng; ++q) mbar_arrive(&empty[(g + q) % NS]);
-  }
+    if (lane < cnt) slot[lane] = sp.m;
+    if (lane + 32 < cnt) slot[32 + lane] = sp.e;
+    __syncwarp();
+    uint32_t sc;
+    q4_lane_block(spans[warp], lane, sc, q);
+    scale = __half2float(__ushort_as_half((unsigned short)sc));
+  };
 
-  // partial y of this CTA
+  // ------------------------------------------------------------- up phase
+  const int ngroups = (n + R - 1) / R;
+  auto load_up = [&](int g, Span (&r)[R][NUP]) {
 #pragma unroll
-  for (int b = 0; b < B; ++b)
+    for (int j = 0; j < R; ++j) {
+      const int i = g * R + j;
+      const int nid = i < n ? ids[i] : -1;
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) {
-      const int u = ct + NCT * c;
-      if (u < nunits) {
-        float4* dst = reinterpret_cast<float4*>(p.part + ((size_t)blockIdx.x * B + b) * p.d +
-                                                (size_t)u * UE);
-#pragma unroll
-        for (int e = 0; e < UE / 4; ++e)
-          dst[e] = make_float4(acc[b][c][4 * e], acc[b][c][4 * e + 1], acc[b][c][4 * e + 2],
-                               acc[b][c][4 * e + 3]);
+      for (int m = 0; m < NUP; ++m) {
+        if (nid >= 0) {
+          load_span((m == 0 ? p.w_act : p.w_up) + (size_t)nid * rb, r[j][m]);
+        } else {
+          r[j][m].m = make_uint4(0, 0, 0, 0);
+          r[j][m].e = make_uint4(0, 0, 0, 0);
+        }
       }
     }
+  };
+  Span ua[R][NUP], ub[R][NUP];
+  if (ngroups > 0) load_up(0, ua);
+  for (int i = t; i < n; i += kQ4Threads)
+    lbias[i] = (p.b_act && ids[i] >= 0) ? p.b_act[ids[i]] : 0.f;
+  float xr[B][32], sx[B];
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
+    float s8 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      widen8<0>(xq[b][k], xr[b] + 8 * k);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s8 += xr[b][8 * k + e];
+    }
+    sx[b] = s8;
+  }
+
+  auto consume_up = [&](int g, const Span (&r)[R][NUP]) {
+    float v[VG];
+#pragma unroll
+    for (int j = 0; j < R; ++j)
+#pragma unroll
+      for (int m = 0; m < NUP; ++m) {
+        float scale;
+        uint32_t q[4];
+        open_span(r[j][m], scale, q);
+        float dq[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) dq[b] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t L = nib_bytes(q[k], false), H = nib_bytes(q[k], true);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float fl = nib16(L, i), fh = nib16(H, i);
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+              dq[b] = fmaf(fl, xr[b][4 * k + i], dq[b]);
+              dq[b] = fmaf(fh, xr[b][4 * k + i + 16], dq[b]);
+            }
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < B; ++b)
+          v[(j * NUP + m) * B + b] = mine ? scale * fmaf(16.f, dq[b], -24.f * sx[b]) : 0.f;
+      }
+    const float tot = warp_reduce_transposed<VG>(v);
+    const int buf = g & 1;
+    if ((lane & ((1 << SHG) - 1)) == 0) red[buf][warp][lane >> SHG] = tot;
+    __syncthreads();
+    if (t < R * B) {
+      const int j = t / B, b = t % B, i = g * R + j;
+      if (i < n) {
+        float act = 0.f, up = 1.f;
+#pragma unroll
+        for (int w = 0; w < kQ4Warps; ++w) act += red[buf][w][(j * NUP) * B + b];
+        if constexpr (ACT == 1) {
+          up = 0.f;
+#pragma unroll
+          for (int w = 0; w < kQ4Warps; ++w) up += red[buf][w][(j * NUP + 1) * B + b];
+        }
+        const float rr = fmaxf(act + lbias[i], 0.f);
+        const float h = ACT == 2 ? rr * rr : rr * up;
+        hs[(size_t)i * B + b] = ids[i] < 0 ? 0.f : h;
+      }
+    }
+  };
+
+  for (int g = 0; g < ngroups; g += 2) {
+    if (g + 1 < ngroups) load_up(g + 1, ub);
+    consume_up(g, ua);
+    if (g + 1 < ngroups) {
+      if (g + 2 < ngroups) load_up(g + 2, ua);
+      consume_up(g + 1, ub);
+    }
+  }
+
+  // ----------------------------------------------------------- down phase
+  auto load_down = [&](int i0, Span (&r)[DH]) {
+#pragma unroll
+    for (int j = 0; j < DH; ++j) {
+      const int i = i0 + j;
+      if (i < n && ids[i] >= 0) {
+        load_span(p.w_dn + (size_t)ids[i] * rb, r[j]);
+      } else {
+        r[j].m = make_uint4(0, 0, 0, 0);
+        r[j].e = make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
+  float acc[B][32], cst[B];
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
+    cst[b] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) acc[b][e] = 0.f;
+  }
+  auto fma_down = [&](int i0, const Span (&r)[DH]) {
+#pragma unroll
+    for (int j = 0; j < DH; ++j) {
+      const int i = i0 + j;
+      if (i < n) {  // CTA-uniform: every lane takes part in the span exchange
+        float scale;
+        uint32_t q[4];
+        open_span(r[j], scale, q);
+        float hsc[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const float hq = hs[(size_t)i * B + b] * scale;  // h * scale
+          hsc[b] = 16.f * hq;
+          cst[b] = fmaf(-24.f, hq, cst[b]);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t L = nib_bytes(q[k], false), H = nib_bytes(q[k], true);
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii) {
+            const float fl = nib16(L, ii), fh = nib16(H, ii);
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+              acc[b][4 * k + ii] = fmaf(hsc[b], fl, acc[b][4 * k + ii]);
+              acc[b][4 * k + ii + 16] = fmaf(hsc[b], fh, acc[b][4 * k + ii + 16]);
+            }
+          }
+        }
+      }
+    }
+  };
+
+  Span d0[DH], d1[DH];
+  load_down(0, d0);  // in flight across the barrier (rows need no h)
+  __syncthreads();   // every h of the slice is in shared memory
+  for (int i0 = 0; i0 < n; i0 += 2 * DH) {
+    load_down(i0 + DH, d1);
+    fma_down(i0, d0);
+    if (i0 + DH < n) {
+      load_down(i0 + 2 * DH, d0);
+      fma_down(i0 + DH, d1);
+    }
+  }
+
+  // partial y of this CTA: columns 32t .. 32t+31
+  if (mine) {
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      float4* dst = reinterpret_cast<float4*>(p.part + ((size_t)blockIdx.x * B + b) * d +
+                                              (size_t)t * 32);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        dst[e] = make_float4(acc[b][4 * e] + cst[b], acc[b][4 * e + 1] + cst[b],
+                             acc[b][4 * e + 2] + cst[b], acc[b][4 * e + 3] + cst[b]);
+    }
+  }
 }
 
 // ------------------------------------------------------ partial reduction
