@@ -331,6 +331,26 @@ cudaError_t pred2_cpl(const pi_predictor* P, const float* a, uint32_t* mask, flo
   return cudaErrorInvalidValue;
 }
 
+// batches of 8+ with 16-bit rows: tensor-core tiles of 16 rows x 8 tokens
+template <int MODE, int WDT, int ACT, int NT>
+cudaError_t launch_rows_mma_nt(const RowsParams& p, int tiles, cudaStream_t st) {
+  constexpr int NUP = (MODE == kModeUp && ACT == 1) ? 2 : 1;
+  const size_t smem = (size_t)kMmaWarps * NUP * NT * 4 * 32 * sizeof(float);
+  return launch(k_rows_mma<MODE, WDT, ACT, NT>, dim3(tiles), dim3(32 * kMmaWarps), smem, st, p);
+}
+
+// one CTA per tile of 16 rows (the upper bound nrows_work; CTAs past the
+// device-side row count return at once)
+template <int MODE, int WDT, int ACT>
+cudaError_t launch_rows_mma(const RowsParams& p, int nrows_work, cudaStream_t st) {
+  const int tiles = std::max(1, (nrows_work + 15) / 16);
+  const int nt = (p.B + 7) / 8;
+  if (nt <= 1) return launch_rows_mma_nt<MODE, WDT, ACT, 1>(p, tiles, st);
+  if (nt <= 2) return launch_rows_mma_nt<MODE, WDT, ACT, 2>(p, tiles, st);
+  if (nt <= 4) return launch_rows_mma_nt<MODE, WDT, ACT, 4>(p, tiles, st);
+  return launch_rows_mma_nt<MODE, WDT, ACT, 8>(p, tiles, st);
+}
+
 template <int DT, int MODE, int BB>
 cudaError_t launch_rows(const RowsParams& p, int nrows_work, cudaStream_t st) {
   const int nsm = num_sms();
@@ -341,6 +361,7 @@ cudaError_t launch_rows(const RowsParams& p, int nrows_work, cudaStream_t st) {
 
 template <int DT, int MODE>
 cudaError_t rows_bb(const RowsParams& p, int nrows_work, cudaStream_t st) {
+  if (MODE == kModePred1 && p.B >= 8) return launch_rows_mma<kModePred1, DT, 0>(p, nrows_work, st);
   if (p.B <= 8) return launch_rows<DT, MODE, 8>(p, nrows_work, st);
   if (p.B <= 32) return launch_rows<DT, MODE, 32>(p, nrows_work, st);
   return launch_rows<DT, MODE, 64>(p, nrows_work, st);
@@ -605,6 +626,8 @@ cudaError_t launch_up_generic(const pi_layer* L, int B, const uint16_t* x, const
   p.len = L->d_model;
   p.B = B;
   const int nsm = num_sms();
+  if constexpr (WDT != 2)
+    if (B >= 8) return launch_rows_mma<kModeUp, WDT, ACT>(p, L->d_ff, st);
   const int blocks = std::min((L->d_ff + 7) / 8, nsm * 8);
   if (B <= 8) return launch(k_rows<kModeUp, WDT, ACT, 8>, dim3(blocks), dim3(256), 0, st, p);
   if (B <= 32) return launch(k_rows<kModeUp, WDT, ACT, 32>, dim3(blocks), dim3(256), 0, st, p);
@@ -683,11 +706,27 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     dp.F = L->d_ff;
     dp.B = B;
     G = down_slices(d, B, num_sms());
-    dim3 grid((d / 8 + 255) / 256, G);
-    switch (L->wdtype) {
-      case PI_F16: e = launch(k_down<0>, grid, dim3(256), 0, st, dp); break;
-      case PI_BF16: e = launch(k_down<1>, grid, dim3(256), 0, st, dp); break;
-      default: e = launch(k_down<2>, grid, dim3(256), 0, st, dp); break;
+    if (L->wdtype != PI_Q4_0 && B % 4 == 0) {
+      // one pass over the rows for all tokens: 64 / BB columns per thread
+      const int BB = B <= 8 ? 8 : B <= 16 ? 16 : B <= 32 ? 32 : 64;
+      const int units = d / (64 / BB);
+      const int gx = (units + 255) / 256;
+      G = std::max(1, std::min(G, 2 * num_sms() / gx));
+      dim3 grid(gx, G);
+      const bool bf = L->wdtype == PI_BF16;
+      switch (BB) {
+        case 8: e = bf ? launch(k_down2<1, 8>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 8>, grid, dim3(256), 0, st, dp); break;
+        case 16: e = bf ? launch(k_down2<1, 16>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 16>, grid, dim3(256), 0, st, dp); break;
+        case 32: e = bf ? launch(k_down2<1, 32>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 32>, grid, dim3(256), 0, st, dp); break;
+        default: e = bf ? launch(k_down2<1, 64>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 64>, grid, dim3(256), 0, st, dp); break;
+      }
+    } else {
+      dim3 grid((d / 8 + 255) / 256, G);
+      switch (L->wdtype) {
+        case PI_F16: e = launch(k_down<0>, grid, dim3(256), 0, st, dp); break;
+        case PI_BF16: e = launch(k_down<1>, grid, dim3(256), 0, st, dp); break;
+        default: e = launch(k_down<2>, grid, dim3(256), 0, st, dp); break;
+      }
     }
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "batched down launch failed: %s", cudaGetErrorString(e));
   }

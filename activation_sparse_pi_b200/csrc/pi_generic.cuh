@@ -86,10 +86,10 @@ __global__ void __launch_bounds__(256) k_rows(RowsParams p) {
 #pragma unroll
       for (int b = 0; b < BB; ++b) acc[m][b] = 0.f;
 
+    if constexpr (WDT == 2) {
 #pragma unroll
-    for (int m = 0; m < NUP; ++m) {
-      const uint8_t* rowp = (m == 0 ? p.w : p.w2nd) + (size_t)nid * rb;
-      if constexpr (WDT == 2) {
+      for (int m = 0; m < NUP; ++m) {
+        const uint8_t* rowp = (m == 0 ? p.w : p.w2nd) + (size_t)nid * rb;
         for (int blk = lane; blk < p.len / 32; blk += 32) {
           const uint16_t* h16 = reinterpret_cast<const uint16_t*>(rowp + (size_t)blk * 18);
           const float sc = __half2float(__ushort_as_half(h16[0]));
@@ -124,28 +124,43 @@ __global__ void __launch_bounds__(256) k_rows(RowsParams p) {
             }
           }
         }
-      } else {
-        for (int c = lane; c < p.len / 8; c += 32) {
-          const uint4 w = __ldg(reinterpret_cast<const uint4*>(rowp + (size_t)c * 16));
+      }
+    } else {
+      // four chunks of each of the neuron's rows in flight per lane; each
+      // widened x chunk serves all of them
+      constexpr int U = 4;
+      const int nch = p.len / 8;
+      const uint8_t* rows[NUP];
 #pragma unroll
-          for (int b = 0; b < BB; ++b) {
-            if (b < B) {
-              if constexpr (MODE == kModePred2) {
-                const float4* ap = reinterpret_cast<const float4*>(p.x32 + (size_t)b * p.len + c * 8);
-                const float4 a0 = __ldg(ap), a1 = __ldg(ap + 1);
-                const float2 f0 = unpack2<WDT>(w.x), f1 = unpack2<WDT>(w.y);
-                const float2 f2 = unpack2<WDT>(w.z), f3 = unpack2<WDT>(w.w);
-                float s = acc[m][b];
-                s = fmaf(f0.x, a0.x, s); s = fmaf(f0.y, a0.y, s);
-                s = fmaf(f1.x, a0.z, s); s = fmaf(f1.y, a0.w, s);
-                s = fmaf(f2.x, a1.x, s); s = fmaf(f2.y, a1.y, s);
-                s = fmaf(f3.x, a1.z, s); s = fmaf(f3.y, a1.w, s);
-                acc[m][b] = s;
-              } else {
-                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x16 + (size_t)b * p.len + c * 8));
+      for (int m = 0; m < NUP; ++m) rows[m] = (m == 0 ? p.w : p.w2nd) + (size_t)nid * rb;
+      for (int c0 = lane; c0 < nch; c0 += 32 * U) {
+        uint4 wq[NUP][U];
+#pragma unroll
+        for (int m = 0; m < NUP; ++m)
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int c = c0 + 32 * u;
+            wq[m][u] = c < nch ? ldg_stream(rows[m] + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int c = c0 + 32 * u;
+          if (c < nch) {
+#pragma unroll
+            for (int b = 0; b < BB; ++b) {
+              if (b < B) {
                 float xf[8];
-                widen8<XDT>(xv, xf);
-                acc[m][b] += dot8<WDT == 2 ? 0 : WDT>(w, xf);
+                if constexpr (MODE == kModePred2) {
+                  const float4* ap = reinterpret_cast<const float4*>(p.x32 + (size_t)b * p.len + c * 8);
+                  const float4 a0 = __ldg(ap), a1 = __ldg(ap + 1);
+                  xf[0] = a0.x; xf[1] = a0.y; xf[2] = a0.z; xf[3] = a0.w;
+                  xf[4] = a1.x; xf[5] = a1.y; xf[6] = a1.z; xf[7] = a1.w;
+                } else {
+                  const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x16 + (size_t)b * p.len + c * 8));
+                  widen8<XDT>(xv, xf);
+                }
+#pragma unroll
+                for (int m = 0; m < NUP; ++m) acc[m][b] += dot8<WDT == 2 ? 0 : WDT>(wq[m][u], xf);
               }
             }
           }
@@ -264,6 +279,275 @@ __global__ void __launch_bounds__(256) k_down(DownParams p) {
       }
     }
   }
+}
+
+// ------------------------------------- batched gathered down, 16-bit, B % 4 == 0
+// One pass over the slice's rows for all tokens: thread t owns CW = 64/BB
+// consecutive columns (so BB x CW = 64 fp32 accumulators), four neurons'
+// index and row loads are in flight at a time, and the h values of a neuron
+// (B floats) are read as float4s that every thread of the CTA shares via L1.
+template <int CW>
+__device__ __forceinline__ void load_cw(const uint8_t* p, uint32_t (&w)[(CW + 1) / 2]) {
+  if constexpr (CW == 8) {
+    const uint4 v = ldg_stream(p);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (CW == 4) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    w[0] = v.x; w[1] = v.y;
+  } else if constexpr (CW == 2) {
+    w[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
+  } else {
+    w[0] = __ldg(reinterpret_cast<const uint16_t*>(p));
+  }
+}
+
+template <int WDT, int BB>
+__global__ void __launch_bounds__(256) k_down2(DownParams p) {
+  constexpr int CW = 64 / BB;          // columns per thread
+  constexpr int NW = (CW + 1) / 2;     // 32-bit words per row piece
+  constexpr int U = 8;                 // neurons in flight
+  pdl_wait();
+  pdl_trigger();
+  int K = *p.count;
+  K = K < 0 ? 0 : (K > p.F ? p.F : K);
+  const int S = gridDim.y;
+  const int k0 = (int)(((long long)K * blockIdx.y) / S);
+  const int k1 = (int)(((long long)K * (blockIdx.y + 1)) / S);
+  const int cu = blockIdx.x * blockDim.x + threadIdx.x;  // unit of CW columns
+  if (cu * CW >= p.d) return;
+  const size_t rb = (size_t)p.d * 2;
+  const int B = p.B;
+  float acc[BB][CW];
+#pragma unroll
+  for (int b = 0; b < BB; ++b)
+#pragma unroll
+    for (int e = 0; e < CW; ++e) acc[b][e] = 0.f;
+  // the next group's neuron ids are requested while this group's rows load
+  int nxt[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) nxt[u] = k0 + u < k1 ? p.idx[k0 + u] : 0;
+  for (int k = k0; k < k1; k += U) {
+    int nid[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = nxt[u];
+      nid[u] = (v < 0 || v >= p.F) ? 0 : v;  // an invalid entry's h is zero
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) nxt[u] = k + U + u < k1 ? p.idx[k + U + u] : 0;
+    uint32_t w[U][NW];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (k + u < k1) load_cw<CW>(p.w_dn + (size_t)nid[u] * rb + (size_t)cu * CW * 2, w[u]);
+      else
+#pragma unroll
+        for (int q = 0; q < NW; ++q) w[u][q] = 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (k + u < k1) {
+        float wf[CW];
+        if constexpr (CW == 1) {
+          wf[0] = WDT == 0 ? __half2float(__ushort_as_half((unsigned short)w[u][0]))
+                           : __uint_as_float(w[u][0] << 16);
+        } else {
+#pragma unroll
+          for (int q = 0; q < NW; ++q) {
+            const float2 f = unpack2<WDT>(w[u][q]);
+            wf[2 * q] = f.x;
+            wf[2 * q + 1] = f.y;
+          }
+        }
+        const float4* hp = reinterpret_cast<const float4*>(p.h + (size_t)(k + u) * B);
+#pragma unroll
+        for (int b4 = 0; b4 < BB / 4; ++b4) {
+          if (4 * b4 < B) {
+            const float4 hv = __ldg(hp + b4);
+            const float hb[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int e = 0; e < CW; ++e) acc[4 * b4 + i][e] = fmaf(hb[i], wf[e], acc[4 * b4 + i][e]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < BB; ++b) {
+    if (b < B) {
+      float* dst = p.part + ((size_t)blockIdx.y * B + b) * p.d + (size_t)cu * CW;
+#pragma unroll
+      for (int e = 0; e < CW; ++e) dst[e] = acc[b][e];
+    }
+  }
+}
+
+// --------------------------------- batched row GEMM on tensor cores (mma.sync)
+// For batches of 8 or more tokens, the rows-times-activations products of the
+// predictor's first layer and of the gathered up projection are small GEMMs:
+// D[16 neurons x 8 tokens] += A[16 x 16] B[16 x 8] with m16n8k16 (fp32
+// accumulate, so products of 16-bit values are exact).  A warp takes a tile
+// of 16 rows and walks the row length in steps of 32 elements.  The
+// contraction index is permuted the same way in A and B so that each lane's
+// A fragment is 16 contiguous bytes of one row and its B fragment 16
+// contiguous bytes of one token: lane (g = lane/4, t = lane%4) loads
+// elements [32s + 8t, 32s + 8t + 8) of rows g and g+8 (words W0..W3) and of
+// token g of each 8-token tile (words X0..X3); k-step 2s uses (W0, W1 | X0,
+// X1), k-step 2s+1 uses (W2, W3 | X2, X3).  Over t = 0..3 the four word
+// slots cover the 32 elements of the step exactly once.
+template <int WDT>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  if constexpr (WDT == 0)
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// MODE kModePred1: rows = W1 (dense), out a[b x r] = relu(. + b1).
+// MODE kModeUp:    rows = idx-gathered activation rows (and W_up for ReGLU),
+//                  out h[k x B].  NT = 8-token tiles (B <= 8 NT).
+// One CTA per tile of 16 rows; its 8 warps split the row length (warp w takes
+// steps [w S/8, (w+1) S/8)), and the 8 partial accumulators are added in warp
+// order through shared memory, so the sum is reproducible.
+constexpr int kMmaWarps = 8;
+
+template <int MODE, int WDT, int ACT, int NT>
+__global__ void __launch_bounds__(32 * kMmaWarps) k_rows_mma(RowsParams p) {
+  constexpr int NUP = (MODE == kModeUp && ACT == 1) ? 2 : 1;
+  constexpr int NV = NUP * NT * 4;  // accumulator values per lane
+  constexpr int U = 4;              // 32-element steps whose loads are in flight together
+  extern __shared__ __align__(16) float part_s[];  // [kMmaWarps][NV][32]
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  int nrows = p.nrows;
+  if (MODE == kModeUp) {
+    const int K = *p.count;
+    nrows = K < 0 ? 0 : (K > p.nrows ? p.nrows : K);
+  }
+  const int tile = blockIdx.x;
+  if (tile * 16 >= nrows) return;  // whole CTA: no barrier is skipped by part of it
+  const int B = p.B;
+  const int len = p.len;
+  const int nsteps = len / 32;
+  const int s_lo = (int)(((long long)nsteps * warp) / kMmaWarps);
+  const int s_hi = (int)(((long long)nsteps * (warp + 1)) / kMmaWarps);
+  const size_t rb = (size_t)len * 2;
+  const uint64_t pol = policy_evict_first();
+
+  int nid[2];
+  bool ok[2];
+#pragma unroll
+  for (int hlf = 0; hlf < 2; ++hlf) {
+    const int row = tile * 16 + g + 8 * hlf;
+    int v = row;
+    bool valid = row < nrows;
+    if (MODE == kModeUp && valid) {
+      v = p.idx[row];
+      if (v < 0 || v >= p.nrows) {
+        if (warp == 0) set_error(kErrBadIndex);
+        valid = false;
+      }
+    }
+    nid[hlf] = valid ? v : 0;
+    ok[hlf] = valid;
+  }
+  float acc[NUP][NT][4];
+#pragma unroll
+  for (int m = 0; m < NUP; ++m)
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[m][n][e] = 0.f;
+
+  for (int s0 = s_lo; s0 < s_hi; s0 += U) {
+    uint4 wa[NUP][U][2];
+#pragma unroll
+    for (int m = 0; m < NUP; ++m)
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          const int s = s0 + u;
+          const uint8_t* row = (m == 0 ? p.w : p.w2nd) + (size_t)nid[hlf] * rb;
+          wa[m][u][hlf] = (s < s_hi && ok[hlf])
+                              ? ldg_stream_hint(row + (size_t)s * 64 + (size_t)t * 16, pol)
+                              : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int s = s0 + u;
+      if (s < s_hi) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          const int tok = n * 8 + g;
+          const uint4 xv = tok < B ? __ldg(reinterpret_cast<const uint4*>(
+                                         p.x16 + (size_t)tok * len + (size_t)s * 32 + t * 8))
+                                   : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int m = 0; m < NUP; ++m) {
+            const uint32_t a0[4] = {wa[m][u][0].x, wa[m][u][1].x, wa[m][u][0].y, wa[m][u][1].y};
+            const uint32_t a1[4] = {wa[m][u][0].z, wa[m][u][1].z, wa[m][u][0].w, wa[m][u][1].w};
+            mma16816<WDT>(acc[m][n], a0, xv.x, xv.y);
+            mma16816<WDT>(acc[m][n], a1, xv.z, xv.w);
+          }
+        }
+      }
+    }
+  }
+
+  // the warps' partial sums, added in warp order
+#pragma unroll
+  for (int m = 0; m < NUP; ++m)
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) part_s[((size_t)warp * NV + (m * NT + n) * 4 + e) * 32 + lane] = acc[m][n][e];
+  __syncthreads();
+  if (warp != 0) return;
+#pragma unroll
+  for (int m = 0; m < NUP; ++m)
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMmaWarps; ++w) v += part_s[((size_t)w * NV + (m * NT + n) * 4 + e) * 32 + lane];
+        acc[m][n][e] = v;
+      }
+
+  // epilogue: c0,c1 -> row g, tokens 2t, 2t+1; c2,c3 -> row g+8
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int hlf = e >> 1;
+      const int row = tile * 16 + g + 8 * hlf;
+      const int tok = n * 8 + 2 * t + (e & 1);
+      if (row < nrows && tok < B) {
+        const float bias = p.bias ? p.bias[nid[hlf]] : 0.f;
+        if constexpr (MODE == kModePred1) {
+          p.out[(size_t)tok * p.nrows + row] = fmaxf(acc[0][n][e] + bias, 0.f);
+        } else {
+          float h = fmaxf(acc[0][n][e] + (ok[hlf] ? bias : 0.f), 0.f);
+          if constexpr (ACT == 1) h *= acc[NUP - 1][n][e];
+          if constexpr (ACT == 2) h *= h;
+          if (!ok[hlf]) h = 0.f;
+          p.out[(size_t)row * B + tok] = h;
+        }
+      }
+    }
 }
 
 }  // namespace pi
