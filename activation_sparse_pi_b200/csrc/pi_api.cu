@@ -707,18 +707,20 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     dp.B = B;
     G = down_slices(d, B, num_sms());
     if (L->wdtype != PI_Q4_0 && B % 4 == 0) {
-      // one pass over the rows for all tokens: 64 / BB columns per thread
-      const int BB = B <= 8 ? 8 : B <= 16 ? 16 : B <= 32 ? 32 : 64;
+      // one pass over the rows per 32 tokens: 64 / BB columns per thread
+      const int BB = B <= 8 ? 8 : B <= 16 ? 16 : 32;
       const int units = d / (64 / BB);
       const int gx = (units + 255) / 256;
       G = std::max(1, std::min(G, 2 * num_sms() / gx));
       dim3 grid(gx, G);
       const bool bf = L->wdtype == PI_BF16;
-      switch (BB) {
-        case 8: e = bf ? launch(k_down2<1, 8>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 8>, grid, dim3(256), 0, st, dp); break;
-        case 16: e = bf ? launch(k_down2<1, 16>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 16>, grid, dim3(256), 0, st, dp); break;
-        case 32: e = bf ? launch(k_down2<1, 32>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 32>, grid, dim3(256), 0, st, dp); break;
-        default: e = bf ? launch(k_down2<1, 64>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 64>, grid, dim3(256), 0, st, dp); break;
+      for (int b0 = 0; b0 < B && e == cudaSuccess; b0 += BB) {
+        dp.b0 = b0;
+        switch (BB) {
+          case 8: e = bf ? launch(k_down2<1, 8>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 8>, grid, dim3(256), 0, st, dp); break;
+          case 16: e = bf ? launch(k_down2<1, 16>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 16>, grid, dim3(256), 0, st, dp); break;
+          default: e = bf ? launch(k_down2<1, 32>, grid, dim3(256), 0, st, dp) : launch(k_down2<0, 32>, grid, dim3(256), 0, st, dp); break;
+        }
       }
     } else {
       dim3 grid((d / 8 + 255) / 256, G);

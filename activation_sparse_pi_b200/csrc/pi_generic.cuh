@@ -212,6 +212,7 @@ struct DownParams {
   const float* h;          // [K x B]
   float* part;             // [gridDim.y x B x d]
   int d, F, B;
+  int b0;                  // k_down2: first token of this pass (B is the row stride of h)
 };
 
 template <int WDT>
@@ -317,6 +318,7 @@ __global__ void __launch_bounds__(256) k_down2(DownParams p) {
   if (cu * CW >= p.d) return;
   const size_t rb = (size_t)p.d * 2;
   const int B = p.B;
+  const int nb = min(BB, B - p.b0);  // tokens of this pass
   float acc[BB][CW];
 #pragma unroll
   for (int b = 0; b < BB; ++b)
@@ -358,10 +360,10 @@ __global__ void __launch_bounds__(256) k_down2(DownParams p) {
             wf[2 * q + 1] = f.y;
           }
         }
-        const float4* hp = reinterpret_cast<const float4*>(p.h + (size_t)(k + u) * B);
+        const float4* hp = reinterpret_cast<const float4*>(p.h + (size_t)(k + u) * B + p.b0);
 #pragma unroll
         for (int b4 = 0; b4 < BB / 4; ++b4) {
-          if (4 * b4 < B) {
+          if (4 * b4 < nb) {
             const float4 hv = __ldg(hp + b4);
             const float hb[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
@@ -375,8 +377,8 @@ __global__ void __launch_bounds__(256) k_down2(DownParams p) {
   }
 #pragma unroll
   for (int b = 0; b < BB; ++b) {
-    if (b < B) {
-      float* dst = p.part + ((size_t)blockIdx.y * B + b) * p.d + (size_t)cu * CW;
+    if (b < nb) {
+      float* dst = p.part + ((size_t)blockIdx.y * B + p.b0 + b) * p.d + (size_t)cu * CW;
 #pragma unroll
       for (int e = 0; e < CW; ++e) dst[e] = acc[b][e];
     }
@@ -423,6 +425,7 @@ constexpr int kMmaWarps = 8;
 
 template <int MODE, int WDT, int ACT, int NT>
 __global__ void __launch_bounds__(32 * kMmaWarps) k_rows_mma(RowsParams p) {
+  static_assert(WDT == 0 || WDT == 1, "16-bit rows");
   constexpr int NUP = (MODE == kModeUp && ACT == 1) ? 2 : 1;
   constexpr int NV = NUP * NT * 4;  // accumulator values per lane
   constexpr int U = 4;              // 32-element steps whose loads are in flight together
