@@ -6,7 +6,7 @@
 // (and W_gate) and W_down^T, with no sparse-format conversion (same page,
 // "Neuronenbewusster Operator").  Here W_down is stored transposed, so a
 // neuron's down-projection column is one contiguous row too, and every
-// gathered read is a single contiguous bulk copy.
+// gathered read streams one contiguous row.
 #pragma once
 #include "pi_predict.cuh"
 
