@@ -71,6 +71,21 @@ def env_rank():
             int(os.environ.get("LOCAL_RANK", 0)))
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time: a step ends when every replica has finished."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(tokens_per_rank, world, ms):
+    """Whole-job throughput: the tokens of all replicas over the slowest time."""
+    return world * tokens_per_rank / (ms / 1e3)
+
+
 def src_sha():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "activation_sparse_pi_b200", "csrc")
@@ -307,12 +322,7 @@ def run_ours(args, rank, world, local):
         e1.record()
         torch.cuda.synchronize()
         barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device="cuda")
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(e0.elapsed_time(e1), world, "cuda")
 
     # ---- headline: graph replay of the step
     g, launches_per_step = step_graph(arr)
@@ -324,8 +334,7 @@ def run_ours(args, rank, world, local):
         ms = time_graph(g, args.steps, 0)
     clocks = clk.summary()
     assert pi.pi_device_error() == 0, "device-side error flagged during the timed region"
-    tokens = world * args.steps * T * B
-    value = tokens / (ms / 1e3)
+    value = job_value(args.steps * T * B, world, ms)
     out_sample = Xw.float().cpu()
     assert torch.isfinite(out_sample).all()
     del g
@@ -397,7 +406,7 @@ def run_ours(args, rank, world, local):
                     pi.pi_sparse_ffn(arr[l], x16, B, idx_all, cnt_all, y, ws)
         dreps = 3
         dms = time_graph(gd, dreps, 1)
-        dense_tps = world * dreps * T * B / (dms / 1e3)
+        dense_tps = job_value(dreps * T * B, world, dms)
         extras["dense"] = {"value": round(dense_tps, 2), "unit": UNIT,
                            "speedup_sparse_over_dense": round(value / dense_tps, 3)}
         del gd
@@ -412,7 +421,7 @@ def run_ours(args, rank, world, local):
         Xw.copy_(X0)
         pi.pi_ffn_stack(arr_o, Xw[0], B, None, cnt_o, ws)
         extras["mode_" + other] = {
-            "value": round(world * max(3, args.steps // 2) * T * B / (oms / 1e3), 2),
+            "value": round(job_value(max(3, args.steps // 2) * T * B, world, oms), 2),
             "unit": UNIT, "mean_active_frac_token0": round(float(cnt_o.float().mean()) / F, 4)}
         del go, layers_o, arr_o
 
@@ -436,13 +445,9 @@ def run_ours(args, rank, world, local):
             e2e_step()
         e1.record()
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t_ = torch.tensor([ems], device="cuda")
-            torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
-            ems = float(t_.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
         nbytes = Xh.numel() * Xh.element_size()
-        extras["e2e"] = {"value": round(world * esteps * T * B / (ems / 1e3), 2), "unit": UNIT,
+        extras["e2e"] = {"value": round(job_value(esteps * T * B, world, ems), 2), "unit": UNIT,
                          "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
                          "steps": esteps, "api": "pi_ffn_stack per token, eager launches"}
 
