@@ -386,9 +386,6 @@ struct PredParams {
   int d, r, F;
 };
 
-#ifndef PI_PRED_PF
-#define PI_PRED_PF 0
-#endif
 constexpr int kPredThreads = 256;
 constexpr int kPredWarps = kPredThreads / 32;
 constexpr int kPredMaxUnits = 64;  // units of 8 rows per CTA
@@ -443,9 +440,6 @@ __global__ void __launch_bounds__(kPredThreads, 2) k_predict(PredParams p) {
   // static biases of this CTA's rows, off the critical path
   if (t < n1) bias1[t] = p.b1 ? p.b1[c + t * G] : 0.f;
   for (int e = t; e < n2 * 8; e += kPredThreads) bias2[e >> 3][e & 7] = p.b2[(size_t)(c + (e >> 3) * G) * 8 + (e & 7)];
-#if PI_PRED_PF == 1
-  if (t < n2) prefetch_l2(p.w2 + (size_t)(c + t * G) * 8 * rb2, (uint32_t)(8 * rb2));
-#endif
 
   pdl_trigger();
   pdl_wait();  // x (or the residual) comes from the previous kernel
@@ -555,9 +549,6 @@ __global__ void __launch_bounds__(kPredThreads, 2) k_predict(PredParams p) {
       dst[k] = (i < n2 && cc < nch2) ? ldg_stream(row + (size_t)cc * 16) : make_uint4(0, 0, 0, 0);
     }
   };
-#if PI_PRED_PF == 2
-  if (t < n2) prefetch_l2(p.w2 + (size_t)(c + t * G) * 8 * rb2, (uint32_t)(8 * rb2));
-#endif
   uint4 wr[P2][CPL];
 #pragma unroll
   for (int q = 0; q < P2; ++q) load2(q, wr[q]);

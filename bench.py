@@ -42,7 +42,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one gathered-FFN launch from an ncu capture, as a ratio to the
 # launch's algorithmic bytes, with the hash of the kernel sources it was taken
 # on (a changed kernel invalidates it).
-TRAFFIC = {"ratio": 1.187, "src_sha": "b4eef40fec96c9d0",
+TRAFFIC = {"ratio": 1.187, "src_sha": "0ab03e39e107de07",
            "profile": "profiles/k_ffn_ldg_k_predict_opt67b_2layer.md"}
 
 
