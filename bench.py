@@ -19,7 +19,7 @@ Also reported on the same GPU:
                tokens copied from pinned host memory and results copied back
   cpu_baseline the fp64 oracle on the host cores (bounded sample)
 
-`--impl reference` times the oracle (the reference for this build) instead.
+`--impl reference` times the fp64 oracle on the host cores instead.
 """
 import argparse
 import hashlib
