@@ -1,8 +1,9 @@
 /*
  * pi.h -- C ABI of the predictor-gated sparse FFN for NVIDIA B200 (sm_100a).
  *
- * The operation is PowerInfer's neuron-aware sparse FFN of a ReLU/ReGLU LLM
- * layer (PowerInfer pages: unite.ai, sections "Adaptive Sparsity-Prädiktoren",
+ * The operation is PowerInfer's neuron-aware sparse FFN of a ReLU, ReGLU or
+ * Squared-ReLU LLM layer (PowerInfer pages: unite.ai, sections "Adaptive
+ * Sparsity-Prädiktoren",
  * "Neuronen-Platzierung und -Verwaltung" and "Neuronenbewusster Operator";
  * machine-heart re-post, Figure 8).  Per token and layer:
  *   1. a low-rank predictor MLP scores every FFN neuron      (pi_predict)
