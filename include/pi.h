@@ -3,9 +3,9 @@
  *
  * The operation is PowerInfer's neuron-aware sparse FFN of a ReLU, ReGLU or
  * Squared-ReLU LLM layer (PowerInfer pages: unite.ai, sections "Adaptive
- * Sparsity-Prädiktoren",
- * "Neuronen-Platzierung und -Verwaltung" and "Neuronenbewusster Operator";
- * machine-heart re-post, Figure 8).  Per token and layer:
+ * Sparsity-Prädiktoren", "Neuronen-Platzierung und -Verwaltung" and
+ * "Neuronenbewusster Operator"; machine-heart re-post, Figure 8).  Per token
+ * and layer:
  *   1. a low-rank predictor MLP scores every FFN neuron      (pi_predict)
  *   2. the neurons predicted active are compacted into an ascending index
  *      list, the union over the batch                        (pi_compact)
