@@ -1,8 +1,15 @@
-"""fp64 CPU oracle (test infrastructure; see pi_oracle's header)."""
-from .pi_oracle import (  # noqa: F401
+"""fp64 CPU oracle of the predictor-gated sparse FFN (test infrastructure).
+
+The oracle is the plain, single-threaded C++ program in pi_oracle.cpp; this
+package exposes it to the tests, the smoke check and the benchmark's CPU legs
+through ctypes (cpp.py).  numpy_xcheck.py is an independent numpy restatement
+kept only as a cross-check pin.  Nothing here is used by the CUDA library.
+"""
+from .cpp import (  # noqa: F401
     RMS_EPS,
-    OracleLayer,
+    CppOracle,
     band,
+    default,
     dense_ffn,
     dequant_q4_0,
     ffn_stack,
@@ -20,3 +27,4 @@ from .pi_oracle import (  # noqa: F401
     widen_bf16,
     widen_f16,
 )
+from .layer import OracleLayer  # noqa: F401

@@ -1,9 +1,10 @@
-"""fp64 CPU oracle of the predictor-gated sparse FFN (test infrastructure).
+"""numpy cross-check of the C++ fp64 oracle (test infrastructure).
 
-This module is the reference the CUDA library is checked against.  It is test
-infrastructure: only the test suite, the package smoke check and the
-benchmark's CPU-baseline leg may import it; the library never calls it and has
-no CPU fallback.  It shares no code with the CUDA path.
+The oracle the CUDA library is checked against is the plain single-threaded
+C++ program in oracle/pi_oracle.cpp.  This module restates the same steps with
+numpy matrix products and serves one purpose: a pin that the two independent
+restatements agree.  Only the test suite imports it; it shares no code with
+the CUDA path or with the C++ oracle.
 
 What it computes, and where the pages state it:
 
@@ -41,10 +42,11 @@ The pages give no formulas.  The readings used here are the plain ones:
 
 Every weight is widened exactly to fp64; all arithmetic is fp64.
 """
-from dataclasses import dataclass
 from typing import Iterable, Optional
 
 import numpy as np
+
+from .layer import OracleLayer
 
 RMS_EPS = 1e-6
 
@@ -125,34 +127,12 @@ def round16(x: np.ndarray, dtype: str) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
-# a layer, with weights kept in their stored form and widened on use
+# a layer's rows, widened on use
 # --------------------------------------------------------------------------
-@dataclass
-class OracleLayer:
-    d_model: int
-    d_ff: int
-    act: str                     # "relu" | "reglu" | "sqrelu"
-    wdtype: str                  # FFN matrices: "f16" | "bf16" | "q4_0"
-    pdtype: str                  # predictor matrices: "f16" | "bf16"
-    w1: np.ndarray               # stored [r x d]
-    b1: Optional[np.ndarray]     # [r] f32/f64 or None
-    w2: np.ndarray               # stored [F x r]
-    b2: np.ndarray               # [F]
-    threshold: float
-    w_up: np.ndarray             # stored rows [F x ...]
-    w_gate: Optional[np.ndarray]
-    w_down_t: np.ndarray
-    b_up: Optional[np.ndarray] = None
-    b_gate: Optional[np.ndarray] = None
-
-    def rows(self, name: str, idx: np.ndarray) -> np.ndarray:
-        """fp64 copies of the given neuron rows of one FFN matrix."""
-        m = getattr(self, name)
-        return widen(m[np.asarray(idx, dtype=np.int64)], self.wdtype, self.d_model)
-
-    @property
-    def rank(self) -> int:
-        return self.w1.shape[0]
+def rows(layer: OracleLayer, name: str, idx: np.ndarray) -> np.ndarray:
+    """fp64 copies of the given neuron rows of one FFN matrix."""
+    m = getattr(layer, name)
+    return widen(np.asarray(m)[np.asarray(idx, dtype=np.int64)], layer.wdtype, layer.d_model)
 
 
 # --------------------------------------------------------------------------
@@ -191,7 +171,7 @@ def neuron_outputs(layer: OracleLayer, x: np.ndarray, idx: np.ndarray) -> np.nda
     """h [B x K]: activation of each listed neuron for each token."""
     x = np.atleast_2d(np.asarray(x, dtype=np.float64))
     idx = np.asarray(idx, dtype=np.int64)
-    up = layer.rows("w_up", idx)
+    up = rows(layer, "w_up", idx)
     if layer.act in ("relu", "sqrelu"):
         pre = x @ up.T
         if layer.b_up is not None:
@@ -199,7 +179,7 @@ def neuron_outputs(layer: OracleLayer, x: np.ndarray, idx: np.ndarray) -> np.nda
         r = np.maximum(pre, 0.0)
         return r if layer.act == "relu" else r * r
     if layer.act == "reglu":
-        gate = layer.rows("w_gate", idx)
+        gate = rows(layer, "w_gate", idx)
         g = x @ gate.T
         if layer.b_gate is not None:
             g = g + np.asarray(layer.b_gate, dtype=np.float64)[idx]
@@ -214,7 +194,7 @@ def masked_ffn(layer: OracleLayer, x: np.ndarray, idx: np.ndarray) -> np.ndarray
     if idx.size == 0:
         return np.zeros((x.shape[0], layer.d_model))
     h = neuron_outputs(layer, x, idx)
-    down = layer.rows("w_down_t", idx)
+    down = rows(layer, "w_down_t", idx)
     return h @ down
 
 

@@ -1,165 +1,121 @@
 """The pins must catch plausible mistakes in the oracle.
 
-Each case swaps one oracle function for a copy with a planted mistake (on the
-CPU, in this process only) and checks that at least one pin then fails.
+Each case copies the C++ oracle's source, plants one mistake in the copy (a
+dropped term, a wrong sign, index or bit field, a transposed operand), compiles
+it into a temporary library on the CPU, points the `oracle` functions at that
+build for the duration of the case, and checks that at least one pin fails.
+The committed oracle is never modified.
 """
-import numpy as np
+import concurrent.futures
+import os
+
 import pytest
 
 import oracle
-import oracle.pi_oracle as po
+import oracle.cpp as ocpp
+from oracle import build as obuild
 from tests import test_oracle_pins as pins
 
-
-def _predict_no_relu(layer, x):
-    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
-    w1 = po.widen(layer.w1, layer.pdtype)
-    w2 = po.widen(layer.w2, layer.pdtype)
-    a = x @ w1.T + (0 if layer.b1 is None else layer.b1)
-    s = a @ w2.T + layer.b2
-    return a, s, s > layer.threshold
-
-
-def _predict_no_b2(layer, x):
-    a, s, _ = _ORIG["predict"](layer, x)
-    s = s - np.asarray(layer.b2)
-    return a, s, s > layer.threshold
-
-
-def _predict_tie_active(layer, x):
-    a, s, _ = _ORIG["predict"](layer, x)
-    return a, s, s >= layer.threshold
-
-
-def _masked_wrong_row(layer, x, idx):
-    idx = np.asarray(idx, dtype=np.int64)
-    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
-    if idx.size == 0:
-        return np.zeros((x.shape[0], layer.d_model))
-    h = po.neuron_outputs(layer, x, idx)
-    down = layer.rows("w_down_t", np.arange(idx.size))   # position, not neuron id
-    return h @ down
-
-
-def _outputs_reglu_swapped(layer, x, idx):
-    if layer.act != "reglu":
-        return _ORIG["neuron_outputs"](layer, x, idx)
-    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
-    up = layer.rows("w_up", idx)
-    gate = layer.rows("w_gate", idx)
-    g = x @ up.T
-    if layer.b_gate is not None:
-        g = g + np.asarray(layer.b_gate)[idx]
-    return np.maximum(g, 0.0) * (x @ gate.T)
-
-
-def _outputs_sqrelu_unsquared(layer, x, idx):
-    if layer.act != "sqrelu":
-        return _ORIG["neuron_outputs"](layer, x, idx)
-    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
-    pre = x @ layer.rows("w_up", idx).T
-    if layer.b_up is not None:
-        pre = pre + np.asarray(layer.b_up)[idx]
-    return np.maximum(pre, 0.0)
-
-
-def _outputs_drop_bias(layer, x, idx):
-    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
-    up = layer.rows("w_up", idx)
-    if layer.act == "relu":
-        return np.maximum(x @ up.T, 0.0)
-    if layer.act == "sqrelu":
-        return np.maximum(x @ up.T, 0.0) ** 2
-    gate = layer.rows("w_gate", idx)
-    return np.maximum(x @ gate.T, 0.0) * (x @ up.T)
-
-
-def _dequant_nibbles_swapped(rows, d_model):
-    rows = np.asarray(rows, dtype=np.uint8)
-    n = rows.shape[0]
-    nb = d_model // 32
-    blk = rows.reshape(n, nb, 18)
-    scale = po.widen_f16(blk[:, :, 0:2].copy().view(np.uint16).reshape(n, nb))
-    qs = blk[:, :, 2:18].astype(np.int64)
-    q = np.concatenate([(qs >> 4) - 8, (qs & 0x0F) - 8], axis=2).astype(np.float64)
-    return (q * scale[:, :, None]).reshape(n, d_model)
-
-
-def _dequant_offset7(rows, d_model):
-    return _ORIG["dequant_q4_0"](rows, d_model) + _scale_rows(rows, d_model)
-
-
-def _scale_rows(rows, d_model):
-    n = rows.shape[0]
-    nb = d_model // 32
-    blk = np.asarray(rows, dtype=np.uint8).reshape(n, nb, 18)
-    scale = po.widen_f16(blk[:, :, 0:2].copy().view(np.uint16).reshape(n, nb))
-    return np.repeat(scale, 32, axis=1)
-
-
-def _union_intersection(mask):
-    mask = np.atleast_2d(np.asarray(mask, dtype=bool))
-    return np.flatnonzero(mask.all(axis=0)).astype(np.int64)
-
-
-def _rms_no_eps(x_resid, adtype):
-    x = np.atleast_2d(np.asarray(x_resid, dtype=np.float64))
-    with np.errstate(invalid="ignore", divide="ignore"):
-        return po.round16(x / np.sqrt(np.mean(x * x, axis=1, keepdims=True)), adtype)
-
-
-def _round_bf16_truncate(x):
-    x = np.asarray(x, dtype=np.float64)
-    m, e = np.frexp(x)
-    return np.ldexp(np.trunc(np.ldexp(m, 8)), e - 8)
-
-
-_ORIG = {k: getattr(po, k) for k in
-         ("predict", "masked_ffn", "neuron_outputs", "dequant_q4_0", "union_index",
-          "rms_cast", "round_bf16")}
-
+# (name, exact text in pi_oracle.cpp, replacement); each text occurs once
 MUTANTS = [
-    ("predict", _predict_no_relu),
-    ("predict", _predict_no_b2),
-    ("predict", _predict_tie_active),
-    ("masked_ffn", _masked_wrong_row),
-    ("neuron_outputs", _outputs_reglu_swapped),
-    ("neuron_outputs", _outputs_drop_bias),
-    ("neuron_outputs", _outputs_sqrelu_unsquared),
-    ("dequant_q4_0", _dequant_nibbles_swapped),
-    ("dequant_q4_0", _dequant_offset7),
-    ("union_index", _union_intersection),
-    ("rms_cast", _rms_no_eps),
-    ("round_bf16", _round_bf16_truncate),
+    ("predict-no-relu", "a[(size_t)b * r + j] = z > 0.0 ? z : 0.0;", "a[(size_t)b * r + j] = z;"),
+    ("predict-no-b2", "z += L->b2[n];", "(void)0;"),
+    ("predict-no-b1", "if (L->b1) z += L->b1[j];", "(void)0;"),
+    ("predict-tie-active", "z > L->threshold ? 1 : 0", "z >= L->threshold ? 1 : 0"),
+    ("predict-x-transposed", "z += w[k] * x[(size_t)b * d + k];", "z += w[k] * x[(size_t)k * B + b];"),
+    ("masked-row-by-position", "widen_row(L->w_down_t, L->wdtype, idx[k], d, row.data());",
+     "widen_row(L->w_down_t, L->wdtype, k, d, row.data());"),
+    ("masked-h-transposed", "const double hb = h[(size_t)b * K + k];",
+     "const double hb = h[(size_t)k * B + b];"),
+    ("reglu-gate-up-swapped",
+     "widen_row(L->w_up, L->wdtype, i, d, up.data());\n    if (L->act == 1) widen_row(L->w_gate, L->wdtype, i, d, gate.data());",
+     "widen_row(L->act == 1 ? L->w_gate : L->w_up, L->wdtype, i, d, up.data());\n    if (L->act == 1) widen_row(L->w_up, L->wdtype, i, d, gate.data());"),
+    ("relu-drop-bias", "if (L->b_up) u += L->b_up[i];", "(void)0;"),
+    ("reglu-drop-bias", "if (L->b_gate) g += L->b_gate[i];", "(void)0;"),
+    ("reglu-no-relu", "v = (g > 0.0 ? g : 0.0) * u;", "v = g * u;"),
+    ("sqrelu-unsquared", "v = L->act == 2 ? rl * rl : rl;", "v = rl;"),
+    ("q4-nibbles-swapped", "const int lo = p[2 + j] & 0x0f;\n      const int hi = p[2 + j] >> 4;",
+     "const int hi = p[2 + j] & 0x0f;\n      const int lo = p[2 + j] >> 4;"),
+    ("q4-offset-7", "out[blk * 32 + j] = (double)(lo - 8) * scale;",
+     "out[blk * 32 + j] = (double)(lo - 7) * scale;"),
+    ("q4-scale-big-endian", "(uint16_t)(p[0] | (p[1] << 8))", "(uint16_t)((p[0] << 8) | p[1])"),
+    ("union-is-intersection",
+     "bool any = false;\n    for (int b = 0; b < B; ++b) any = any || mask[(size_t)b * F + n] != 0;",
+     "bool any = true;\n    for (int b = 0; b < B; ++b) any = any && mask[(size_t)b * F + n] != 0;"),
+    ("rms-no-eps", "std::sqrt(ss / d + 1e-6)", "std::sqrt(ss / d)"),
+    ("rms-divisor", "std::sqrt(ss / d + 1e-6)", "std::sqrt(ss / (d - 1) + 1e-6)"),
+    ("round-truncates", "std::nearbyint(std::ldexp(ax, -qe))", "std::trunc(std::ldexp(ax, -qe))"),
+    ("round-ties-away", "std::nearbyint(std::ldexp(ax, -qe))", "std::round(std::ldexp(ax, -qe))"),
+    ("bf16-exponent-shift-8", "std::ldexp((double)(128 + m), e - 134)",
+     "std::ldexp((double)(128 + m), e - 126)"),
+    ("bf16-read-as-f16", "out[k] = dtype == 0 ? widen_f16_bits(p[k]) : widen_bf16_bits(p[k]);",
+     "out[k] = widen_f16_bits(p[k]);"),
+    ("bf16-fraction-7-as-8", "const int m = b & 0x7f;\n  double v;\n  if (e == 0) {\n    v = std::ldexp((double)m, -133);",
+     "const int m = b & 0xff;\n  double v;\n  if (e == 0) {\n    v = std::ldexp((double)m, -133);"),
+    ("f16-subnormal-scale", "v = std::ldexp((double)m, -24);", "v = std::ldexp((double)m, -25);"),
+    ("f16-bias-off-by-one", "std::ldexp((double)(1024 + m), e - 25)",
+     "std::ldexp((double)(1024 + m), e - 24)"),
 ]
 
 PIN_CASES = [
-    (pins.test_predict_and_ffn_brute_force, dict(act="relu", shape=(16, 8, 4))),
-    (pins.test_predict_and_ffn_brute_force, dict(act="reglu", shape=(48, 16, 6))),
-    (pins.test_every_subset_closed_form, dict(act="relu")),
-    (pins.test_every_subset_closed_form, dict(act="reglu")),
-    (pins.test_predict_and_ffn_brute_force, dict(act="sqrelu", shape=(16, 8, 4))),
+    (pins.test_predict_and_ffn_brute_force, dict(act="relu", shape=(16, 8, 4), wdtype="f16")),
+    (pins.test_predict_and_ffn_brute_force, dict(act="reglu", shape=(48, 16, 6), wdtype="bf16")),
+    (pins.test_predict_and_ffn_brute_force, dict(act="sqrelu", shape=(16, 8, 4), wdtype="f16")),
+    (pins.test_predict_and_ffn_brute_force, dict(act="relu", shape=(64, 12, 8), wdtype="q4_0")),
+    (pins.test_every_subset_closed_form, dict(act="relu", wdtype="f16")),
+    (pins.test_every_subset_closed_form, dict(act="reglu", wdtype="bf16")),
     (pins.test_tie_is_inactive, {}),
     (pins.test_fig8_worked_example, {}),
     (pins.test_union_index_brute_force, {}),
     (pins.test_predictor_closed_form_pm_construction, {}),
     (pins.test_measured_sparsity_matches_profile, {}),
     (pins.test_q4_0_golden_block, {}),
+    (pins.test_round_f16_ties_and_library, {}),
     (pins.test_round_bf16_ties_and_library, {}),
+    (pins.test_round_overflow_and_subnormal_ties, {}),
     (pins.test_rms_cast_special_cases, {}),
     (pins.test_stack_brute_force, {}),
+    (pins.test_widen_bf16_hand_patterns, {}),
+    (pins.test_widen_f16_hand_patterns, {}),
 ]
 
 
-@pytest.mark.parametrize("name,fn", MUTANTS, ids=[f"{n}:{f.__name__}" for n, f in MUTANTS])
-def test_planted_mistake_fails_a_pin(monkeypatch, name, fn):
-    monkeypatch.setattr(po, name, fn)
-    if hasattr(oracle, name):
-        monkeypatch.setattr(oracle, name, fn)
-    caught = []
+def _mutated_source(old, new):
+    src = open(obuild.SRC).read()
+    assert src.count(old) == 1, f"mutation anchor must occur once: {old!r}"
+    return src.replace(old, new)
+
+
+@pytest.fixture(scope="module")
+def mutant_libs(tmp_path_factory):
+    d = tmp_path_factory.mktemp("oracle_mutants")
+
+    def make(m):
+        name, old, new = m
+        src = os.path.join(d, f"{name}.cpp")
+        with open(src, "w") as f:
+            f.write(_mutated_source(old, new))
+        return name, obuild.compile_source(src, os.path.join(d, f"lib_{name}.so"))
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
+        return dict(ex.map(make, MUTANTS))
+
+
+def test_unmutated_oracle_passes_every_pin_case():
+    for case, kw in PIN_CASES:
+        case(**kw)
+
+
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+def test_planted_mistake_fails_a_pin(monkeypatch, mutant_libs, name):
+    mut = ocpp.CppOracle(mutant_libs[name])
+    for fn in ocpp.API:
+        monkeypatch.setattr(oracle, fn, getattr(mut, fn))
+    caught = None
     for case, kw in PIN_CASES:
         try:
             case(**kw)
-        except (AssertionError, ValueError, FloatingPointError) as e:  # noqa: PERF203
-            caught.append(case.__name__)
-    assert caught, f"no pin caught the planted mistake {fn.__name__}"
+        except (AssertionError, ValueError, FloatingPointError):
+            caught = case.__name__
+            break
+    assert caught, f"no pin caught the planted mistake {name}"

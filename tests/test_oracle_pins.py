@@ -64,32 +64,90 @@ def f16_round_py(v):
 
 
 # ---------------------------------------------------------------------------
-# a tiny random layer with fp16-exact weights
+# stored-weight decoding in plain Python (struct), independent of the oracle
 # ---------------------------------------------------------------------------
-def tiny_layer(rng, d, F, r, act, tau=0.0, bias=True):
-    def h16(shape, std):
-        return (rng.standard_normal(shape) * std).astype(np.float16)
+def f16_py(bits):
+    return struct.unpack("<e", int(bits).to_bytes(2, "little"))[0]
 
-    W1 = h16((r, d), 0.4)
-    W2 = h16((F, r), 0.4)
-    Wup = h16((F, d), 0.3)
-    Wgate = h16((F, d), 0.3) if act == "reglu" else None
-    Wdt = h16((F, d), 0.3)
+
+def bf16_py(bits):
+    """bfloat16 bits are the top half of an IEEE binary32."""
+    return struct.unpack("<f", (int(bits) << 16).to_bytes(4, "little"))[0]
+
+
+def q4_0_row_py(row, d):
+    """One Q4_0 row (d/32 blocks of 18 bytes) decoded byte by byte."""
+    out = []
+    for blk in range(d // 32):
+        b = bytes(row[18 * blk: 18 * blk + 18])
+        scale = struct.unpack("<e", b[0:2])[0]
+        lo = [((b[2 + j] & 15) - 8) * scale for j in range(16)]
+        hi = [((b[2 + j] >> 4) - 8) * scale for j in range(16)]
+        out += lo + hi
+    return out
+
+
+def decode_py(bits, dtype, d=None):
+    bits = np.asarray(bits)
+    if dtype == "q4_0":
+        return [q4_0_row_py(r.tolist(), d) for r in bits]
+    f = f16_py if dtype == "f16" else bf16_py
+    return [[f(v) for v in row] for row in bits.tolist()]
+
+
+def bf16_bits(x):
+    """float32 values -> bfloat16 bit patterns (library round-to-nearest-even)."""
+    t = torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def q4_0_pack(rng, F, d, std):
+    """Random Q4_0 rows: random nibbles and positive/negative fp16 scales."""
+    nb = d // 32
+    rows = np.zeros((F, nb * 18), dtype=np.uint8)
+    for i in range(F):
+        for blk in range(nb):
+            scale = np.float16(std / 8 * rng.uniform(0.5, 1.5) * rng.choice([-1, 1]))
+            q = rng.integers(0, 16, 32)
+            b = bytearray(np.array([scale]).view(np.uint8).tobytes())
+            b += bytes(int(q[j]) | (int(q[j + 16]) << 4) for j in range(16))
+            rows[i, 18 * blk: 18 * blk + 18] = np.frombuffer(bytes(b), dtype=np.uint8)
+    return rows
+
+
+# ---------------------------------------------------------------------------
+# a tiny random layer with weights exact in their stored type
+# ---------------------------------------------------------------------------
+def tiny_layer(rng, d, F, r, act, tau=0.0, bias=True, wdtype="f16", pdtype=None):
+    pdtype = pdtype or ("bf16" if wdtype == "bf16" else "f16")
+
+    def store(shape, std, dt):
+        x = rng.standard_normal(shape) * std
+        if dt == "f16":
+            return x.astype(np.float16).view(np.uint16)
+        if dt == "bf16":
+            return bf16_bits(x)
+        return q4_0_pack(rng, shape[0], shape[1], std)
+
+    W1 = store((r, d), 0.4, pdtype)
+    W2 = store((F, r), 0.4, pdtype)
+    Wup = store((F, d), 0.3, wdtype)
+    Wgate = store((F, d), 0.3, wdtype) if act == "reglu" else None
+    Wdt = store((F, d), 0.3, wdtype)
     b1 = rng.standard_normal(r).astype(np.float32)
     b2 = rng.standard_normal(F).astype(np.float32)
     bact = (rng.standard_normal(F) * 0.5).astype(np.float32) if bias else None
     L = oracle.OracleLayer(
-        d_model=d, d_ff=F, act=act, wdtype="f16", pdtype="f16",
-        w1=W1.view(np.uint16), b1=b1, w2=W2.view(np.uint16), b2=b2, threshold=tau,
-        w_up=Wup.view(np.uint16), w_gate=None if Wgate is None else Wgate.view(np.uint16),
-        w_down_t=Wdt.view(np.uint16),
+        d_model=d, d_ff=F, act=act, wdtype=wdtype, pdtype=pdtype,
+        w1=W1, b1=b1, w2=W2, b2=b2, threshold=tau,
+        w_up=Wup, w_gate=Wgate, w_down_t=Wdt,
         b_up=bact if act != "reglu" else None, b_gate=bact if act == "reglu" else None,
     )
     lists = dict(
-        W1=W1.astype(float).tolist(), W2=W2.astype(float).tolist(),
-        Wup=Wup.astype(float).tolist(),
-        Wgate=None if Wgate is None else Wgate.astype(float).tolist(),
-        Wdt=Wdt.astype(float).tolist(), b1=b1.astype(float).tolist(),
+        W1=decode_py(W1, pdtype), W2=decode_py(W2, pdtype),
+        Wup=decode_py(Wup, wdtype, d),
+        Wgate=None if Wgate is None else decode_py(Wgate, wdtype, d),
+        Wdt=decode_py(Wdt, wdtype, d), b1=b1.astype(float).tolist(),
         b2=b2.astype(float).tolist(),
         bup=bact.astype(float).tolist() if (bias and act != "reglu") else None,
         bgate=bact.astype(float).tolist() if (bias and act == "reglu") else None,
@@ -97,8 +155,11 @@ def tiny_layer(rng, d, F, r, act, tau=0.0, bias=True):
     return L, lists
 
 
-def tokens16(rng, B, d):
-    return rng.standard_normal((B, d)).astype(np.float16).astype(np.float64)
+def tokens16(rng, B, d, adtype="f16"):
+    x = rng.standard_normal((B, d))
+    if adtype == "bf16":
+        return np.array(decode_py(bf16_bits(x), "bf16"))
+    return x.astype(np.float16).astype(np.float64)
 
 
 # ---------------------------------------------------------------------------
@@ -106,11 +167,14 @@ def tokens16(rng, B, d):
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("act", ["relu", "reglu", "sqrelu"])
 @pytest.mark.parametrize("shape", [(16, 8, 4), (48, 16, 6), (64, 12, 8)])
-def test_predict_and_ffn_brute_force(act, shape):
+@pytest.mark.parametrize("wdtype", ["f16", "bf16", "q4_0"])
+def test_predict_and_ffn_brute_force(act, shape, wdtype):
     d, F, r = shape
+    if wdtype == "q4_0":
+        d = 32 * ((d + 31) // 32)
     rng = np.random.default_rng(11 + d + F)
-    L, P = tiny_layer(rng, d, F, r, act, tau=0.3)
-    x = tokens16(rng, 3, d)
+    L, P = tiny_layer(rng, d, F, r, act, tau=0.3, wdtype=wdtype)
+    x = tokens16(rng, 3, d, L.pdtype)
     a, s, m = oracle.predict(L, x)
     for b in range(3):
         ab, sb, mb = bf_predict(P["W1"], P["b1"], P["W2"], P["b2"], x[b].tolist(), 0.3)
@@ -118,6 +182,7 @@ def test_predict_and_ffn_brute_force(act, shape):
         np.testing.assert_allclose(s[b], sb, rtol=1e-12, atol=1e-12)
         assert list(m[b]) == mb
     idx = oracle.union_index(m)
+    assert 0 < idx.size < F
     y = oracle.masked_ffn(L, x, idx)
     yd = oracle.dense_ffn(L, x)
     for b in range(3):
@@ -130,14 +195,15 @@ def test_predict_and_ffn_brute_force(act, shape):
 
 
 @pytest.mark.parametrize("act", ["relu", "reglu", "sqrelu"])
-def test_every_subset_closed_form(act):
+@pytest.mark.parametrize("wdtype", ["f16", "bf16"])
+def test_every_subset_closed_form(act, wdtype):
     """Every index set I of an F = 8 layer: y(I) = y_dense - sum over
     support-minus-I of h_i W_down^T[i]."""
     d, F, r = 24, 8, 4
     for seed in range(100):  # first seed whose token has both zero and nonzero h
         rng = np.random.default_rng(seed)
-        L, P = tiny_layer(rng, d, F, r, act)
-        x = tokens16(rng, 1, d)[0]
+        L, P = tiny_layer(rng, d, F, r, act, wdtype=wdtype)
+        x = tokens16(rng, 1, d, L.pdtype)[0]
         xl = x.tolist()
         h = [bf_h(act, P["Wup"], P["Wgate"], P["bup"], P["bgate"], xl, i) for i in range(F)]
         if 2 <= sum(v != 0.0 for v in h) <= F - 2:
@@ -382,3 +448,114 @@ def test_stack_brute_force():
         y = bf_y("relu", P["Wup"], None, P["Wdt"], P["bup"], None, xl, idx)
         x = [a + b for a, b in zip(x, y)]
     np.testing.assert_allclose(out[0], x, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# widening of stored 16-bit weights, from hand-written bit patterns
+# ---------------------------------------------------------------------------
+def _same(a, b):
+    """Equal as numbers and in sign (so -0.0 differs from 0.0)."""
+    return a == b and math.copysign(1.0, a) == math.copysign(1.0, b)
+
+
+def test_widen_bf16_hand_patterns():
+    """bfloat16: 1 sign, 8 exponent (bias 127), 7 fraction bits."""
+    cases = {
+        0x0000: 0.0, 0x8000: -0.0,
+        0x3F80: 1.0, 0xBF80: -1.0, 0x4000: 2.0, 0x3FC0: 1.5, 0x3F81: 1.0 + 2.0**-7,
+        0xC2F7: -123.5,                        # -(1 + 119/128) * 2^6
+        0x7F7F: (2.0 - 2.0**-7) * 2.0**127,    # largest finite
+        0xFF7F: -(2.0 - 2.0**-7) * 2.0**127,
+        0x0080: 2.0**-126,                     # smallest normal
+        0x0001: 2.0**-133,                     # smallest subnormal
+        0x007F: 127 * 2.0**-133,               # largest subnormal
+        0x7F80: math.inf, 0xFF80: -math.inf,
+    }
+    got = oracle.widen_bf16(np.array(list(cases), dtype=np.uint16))
+    for (bits, want), g in zip(cases.items(), got.tolist()):
+        assert _same(g, want), (hex(bits), g, want)
+    assert np.isnan(oracle.widen_bf16(np.array([0x7FC0], dtype=np.uint16)))[0]
+
+
+def test_widen_f16_hand_patterns():
+    """IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits."""
+    cases = {
+        0x0000: 0.0, 0x8000: -0.0, 0x3C00: 1.0, 0xC000: -2.0, 0x3E00: 1.5,
+        0x3C01: 1.0 + 2.0**-10, 0x7BFF: 65504.0, 0xFBFF: -65504.0,
+        0x0400: 2.0**-14, 0x0001: 2.0**-24, 0x03FF: 1023 * 2.0**-24,
+        0x7C00: math.inf, 0xFC00: -math.inf,
+    }
+    got = oracle.widen_f16(np.array(list(cases), dtype=np.uint16))
+    for (bits, want), g in zip(cases.items(), got.tolist()):
+        assert _same(g, want), (hex(bits), g, want)
+
+
+def test_widen_every_pattern_against_struct():
+    """All 65536 patterns of both types against the struct module's decoders."""
+    bits = np.arange(65536, dtype=np.uint32)
+    f16 = oracle.widen_f16(bits.astype(np.uint16))
+    bf = oracle.widen_bf16(bits.astype(np.uint16))
+    with np.errstate(invalid="ignore"):  # signalling NaN patterns
+        ref16 = np.frombuffer(bits.astype("<u2").tobytes(), dtype="<f2").astype(np.float64)
+        refbf = np.frombuffer((bits << 16).astype("<u4").tobytes(), dtype="<f4").astype(np.float64)
+    for got, ref in ((f16, ref16), (bf, refbf)):
+        nan = np.isnan(ref)
+        assert np.array_equal(np.isnan(got), nan)
+        assert np.array_equal(got[~nan], ref[~nan])
+        assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+    for b in (0x1234, 0x8001, 0xBEEF, 0x3555):
+        assert f16[b] == f16_py(b) and bf[b] == bf16_py(b)
+
+
+def test_widen_then_round_is_identity():
+    """Every finite pattern survives widening followed by rounding back."""
+    bits = np.arange(65536, dtype=np.uint16)
+    bf = oracle.widen_bf16(bits)
+    f16 = oracle.widen_f16(bits)
+    for v, rnd in ((bf, oracle.round_bf16), (f16, oracle.round_f16)):
+        fin = np.isfinite(v)
+        back = rnd(v[fin])
+        assert np.array_equal(back, v[fin])
+        assert np.array_equal(np.signbit(back), np.signbit(v[fin]))
+
+
+# ---------------------------------------------------------------------------
+# rounding at the edges of the formats
+# ---------------------------------------------------------------------------
+def test_round_overflow_and_subnormal_ties():
+    f16 = oracle.round_f16(np.array([
+        65504.0, 65519.99, 65520.0, -70000.0,     # largest finite, below / at the tie to inf
+        2.0**-25, 3 * 2.0**-25, 1.4 * 2.0**-24,   # subnormal ties to even, nearest
+        2.0**-14 - 2.0**-25,                      # rounds up into the normal range
+    ]))
+    assert f16.tolist() == [65504.0, 65504.0, math.inf, -math.inf,
+                            0.0, 2.0**-23, 2.0**-24, 2.0**-14]
+    big = (2.0 - 2.0**-8) * 2.0**127
+    bf = oracle.round_bf16(np.array([
+        big * (1 - 2.0**-30), big, 2.0**-134, 3 * 2.0**-134, 2.0**-126 * (1 + 2.0**-8),
+    ]))
+    assert bf.tolist() == [(2.0 - 2.0**-7) * 2.0**127, math.inf, 0.0, 2.0**-132, 2.0**-126]
+
+
+# ---------------------------------------------------------------------------
+# cross-check: an independent numpy restatement agrees with the C++ oracle
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("act", ["relu", "reglu", "sqrelu"])
+@pytest.mark.parametrize("wdtype", ["f16", "bf16", "q4_0"])
+def test_numpy_restatement_agrees(act, wdtype):
+    import oracle.numpy_xcheck as nx
+    rng = np.random.default_rng(40 + len(act) + len(wdtype))
+    d, F, r = 64, 40, 16
+    L, _ = tiny_layer(rng, d, F, r, act, tau=0.1, wdtype=wdtype)
+    x = tokens16(rng, 5, d, L.pdtype)
+    a1, s1, m1 = oracle.predict(L, x)
+    a2, s2, m2 = nx.predict(L, x)
+    np.testing.assert_allclose(a1, a2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(s1, s2, rtol=1e-12, atol=1e-13)
+    assert np.array_equal(m1, m2)
+    assert np.array_equal(oracle.union_index(m1), nx.union_index(m2))
+    I = oracle.union_index(m1)
+    np.testing.assert_allclose(oracle.masked_ffn(L, x, I), nx.masked_ffn(L, x, I),
+                               rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(oracle.rms_cast(x * 3.0, L.pdtype), nx.rms_cast(x * 3.0, L.pdtype))
+    assert np.array_equal(oracle.widen(L.w_up, wdtype, d), nx.widen(L.w_up, wdtype, d))
