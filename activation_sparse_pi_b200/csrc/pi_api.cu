@@ -6,6 +6,7 @@
 // kernel before it; each kernel waits (griddepcontrol.wait) before it touches
 // that kernel's results.
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <atomic>
@@ -19,6 +20,7 @@
 
 #include "../../include/pi.h"
 #include "pi_generic.cuh"
+#include "pi_umma.cuh"
 
 using namespace pi;
 
@@ -642,6 +644,127 @@ cudaError_t up_generic_act(const pi_layer* L, int B, const uint16_t* x, const in
   return launch_up_generic<WDT, 0>(L, B, x, idx, count, h, st);
 }
 
+// ------------------------------------------------- tensor-core batched path
+// Batches of at least kUmmaMinBatch tokens with 16-bit weights run the
+// gathered up and down projections as tcgen05 GEMMs (pi_umma.cuh); their
+// operands are described to the copy engine by tensor maps built here.
+constexpr int kUmmaMinBatch = 8;
+
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// A row-major [rows x inner] tensor of 16-bit values, read in boxes of
+// box_inner x box_rows with the 128-byte swizzle; rows and columns outside the
+// tensor read as zeros.
+bool make_tmap16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool umma_ok(const pi_layer* L, int B) {
+  return (L->wdtype == PI_F16 || L->wdtype == PI_BF16) && B >= kUmmaMinBatch && B <= 64 &&
+         L->d_model % kUmmaM == 0 && tmap_encoder() != nullptr;
+}
+
+// pipeline stages that fit two CTAs per SM (at least 2, at most 6)
+constexpr int umma_ns(int stage_bytes) {
+  return (110 * 1024) / stage_bytes < 2 ? 2 : (110 * 1024) / stage_bytes > 6 ? 6
+                                              : (110 * 1024) / stage_bytes;
+}
+
+template <int DT, int ACT, int N>
+cudaError_t launch_umma_up_n(const pi_layer* L, const CUtensorMap& ta, const CUtensorMap& ta2,
+                             const CUtensorMap& tx, const UmmaParams& p, cudaStream_t st) {
+  constexpr int NMAT = ACT == 1 ? 2 : 1;
+  constexpr int STAGE = umma_up_stage<NMAT, N>();
+  constexpr int NS = umma_ns(STAGE);
+  const int tiles = (L->d_ff + kUmmaM - 1) / kUmmaM;
+  return launch(k_umma_up<DT, ACT, N, NS>, dim3(tiles), dim3(kUmmaThreads),
+                (size_t)NS * STAGE + 1024, st, ta, ta2, tx, p);
+}
+
+template <int DT, int N>
+cudaError_t launch_umma_down_n(const pi_layer* L, int S, const CUtensorMap& tw,
+                               const CUtensorMap& th, const CUtensorMap& tl, const UmmaParams& p,
+                               cudaStream_t st) {
+  constexpr int STAGE = umma_down_stage<N>();
+  constexpr int NS = umma_ns(STAGE);
+  return launch(k_umma_down<DT, N, NS>, dim3(L->d_model / kUmmaM, S), dim3(kUmmaThreads),
+                (size_t)NS * STAGE + 1024, st, tw, th, tl, p);
+}
+
+template <int DT, int ACT>
+cudaError_t umma_up_act(const pi_layer* L, int N, const CUtensorMap& ta, const CUtensorMap& ta2,
+                        const CUtensorMap& tx, const UmmaParams& p, cudaStream_t st) {
+  switch (N) {
+    case 16: return launch_umma_up_n<DT, ACT, 16>(L, ta, ta2, tx, p, st);
+    case 32: return launch_umma_up_n<DT, ACT, 32>(L, ta, ta2, tx, p, st);
+    case 48: return launch_umma_up_n<DT, ACT, 48>(L, ta, ta2, tx, p, st);
+    default: return launch_umma_up_n<DT, ACT, 64>(L, ta, ta2, tx, p, st);
+  }
+}
+
+template <int DT>
+cudaError_t umma_ffn(const pi_layer* L, int B, const uint16_t* x, const int32_t* idx,
+                     const int32_t* count, uint16_t* hh, uint16_t* hl, float* part, int S,
+                     cudaStream_t st) {
+  const int d = L->d_model, F = L->d_ff;
+  const int N = (B + 15) / 16 * 16;
+  const bool reglu = L->act == PI_REGLU;
+  CUtensorMap ta, ta2, tx, tw, th, tl;
+  const uint64_t rb = (uint64_t)d * 2;
+  if (!make_tmap16(&ta, reglu ? L->w_gate : L->w_up, d, F, rb, kUmmaK, 1) ||
+      !make_tmap16(&ta2, L->w_up, d, F, rb, kUmmaK, 1) ||
+      !make_tmap16(&tx, x, d, B, rb, kUmmaK, N) ||
+      !make_tmap16(&tw, L->w_down_t, d, F, rb, kUmmaK, 1) ||
+      !make_tmap16(&th, hh, F, B, (uint64_t)F * 2, kUmmaK, N) ||
+      !make_tmap16(&tl, hl, F, B, (uint64_t)F * 2, kUmmaK, N))
+    return cudaErrorInvalidValue;
+  UmmaParams p{};
+  p.idx = idx;
+  p.count = count;
+  p.bias = reglu ? L->b_gate : L->b_up;
+  p.hh = hh;
+  p.hl = hl;
+  p.part = part;
+  p.d = d;
+  p.F = F;
+  p.B = B;
+  cudaError_t e = L->act == PI_REGLU ? umma_up_act<DT, 1>(L, N, ta, ta2, tx, p, st)
+                : L->act == PI_SQRELU ? umma_up_act<DT, 2>(L, N, ta, ta2, tx, p, st)
+                                      : umma_up_act<DT, 0>(L, N, ta, ta2, tx, p, st);
+  if (e != cudaSuccess) return e;
+  switch (N) {
+    case 16: return launch_umma_down_n<DT, 16>(L, S, tw, th, tl, p, st);
+    case 32: return launch_umma_down_n<DT, 32>(L, S, tw, th, tl, p, st);
+    case 48: return launch_umma_down_n<DT, 48>(L, S, tw, th, tl, p, st);
+    default: return launch_umma_down_n<DT, 64>(L, S, tw, th, tl, p, st);
+  }
+}
+
+// neuron slices of the tensor-core down projection: about two CTAs per SM
+int umma_slices(int d, int B, int nsm) {
+  const int tiles = d / kUmmaM;
+  return std::max(1, std::min(down_slices(d, B, nsm), (2 * nsm) / tiles));
+}
+
 // Records a caller's timing event on the stream; under stream capture it
 // becomes an external event-record node, so every graph launch records it.
 cudaError_t record_event(void* ev, cudaStream_t st) {
@@ -686,6 +809,17 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     }
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "fused FFN launch failed: %s", cudaGetErrorString(e));
     G = ffn_grid(B);
+  } else if (umma_ok(L, B)) {
+    if (src.mask) return fail(PI_ERR_UNSUPPORTED, "mask-driven FFN needs the fused kernel");
+    uint16_t* hh = reinterpret_cast<uint16_t*>(ws + w.h);
+    uint16_t* hl = hh + (size_t)L->d_ff * B;
+    G = umma_slices(d, B, num_sms());
+    const cudaError_t e =
+        L->wdtype == PI_BF16
+            ? umma_ffn<1>(L, B, x, src.idx, src.count, hh, hl, part, G, st)
+            : umma_ffn<0>(L, B, x, src.idx, src.count, hh, hl, part, G, st);
+    if (e != cudaSuccess)
+      return fail(PI_ERR_CUDA, "tensor-core FFN launch failed: %s", cudaGetErrorString(e));
   } else {
     if (src.mask) return fail(PI_ERR_UNSUPPORTED, "mask-driven FFN needs the fused kernel");
     float* h = reinterpret_cast<float*>(ws + w.h);
@@ -897,9 +1031,9 @@ int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_re
 // whole device, a latency-bound loop in which an allocation (which may wait
 // for the device) is not allowed, or code that only holds weights and
 // activations -- get the gathered FFN without supplying a workspace.
-// The scratch lives in g_static_scratch; its address is looked up once per
-// device (the first call on a device does this, so make it before any stream
-// capture).  Nothing in the scratch has to start at zero: every CTA writes its
+// The scratch lives in g_static_scratch; its address is looked up at set-up
+// (the first call on a device, which must come before any stream capture) and
+// refreshed on every uncaptured call.  Nothing in the scratch has to start at zero: every CTA writes its
 // whole partial plane, and h is written for every listed neuron before it is
 // read.  Calls whose work overlaps on one device race on the scratch.
 int32_t pi_sparse_ffn_static(const pi_layer* layer, const void* x, int32_t batch,
@@ -928,12 +1062,22 @@ int32_t pi_sparse_ffn_static(const pi_layer* layer, const void* x, int32_t batch
   if (dev < 0 || dev >= kMaxDevices)
     return fail(PI_ERR_UNSUPPORTED, "device ordinal %d: the fixed scratch supports 0..%d", dev,
                 kMaxDevices - 1);
+  // The address is looked up with this device current: at set-up (the first
+  // call on the device), and again on every call made outside stream capture,
+  // so a device reset (which reloads the module at another address) cannot
+  // leave a stale pointer behind.  Under capture the set-up value is used.
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  PI_CUDA(cudaStreamIsCapturing(st, &cs));
   static std::mutex mu;
   static uint8_t* base[kMaxDevices] = {};
   uint8_t* ws = nullptr;
   {
     std::lock_guard<std::mutex> lk(mu);
-    if (!base[dev]) {
+    if (cs == cudaStreamCaptureStatusNone || !base[dev]) {
+      if (cs != cudaStreamCaptureStatusNone)
+        return fail(PI_ERR_INVALID_ARG,
+                    "pi_sparse_ffn_static: the first call on a device must not be captured");
       void* ptr = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
       if (e != cudaSuccess)
@@ -944,8 +1088,7 @@ int32_t pi_sparse_ffn_static(const pi_layer* layer, const void* x, int32_t batch
     ws = base[dev];
   }
   FfnSrc src{idx, count, nullptr, 0, nullptr, nullptr};
-  return ffn_impl(layer, batch, static_cast<const uint16_t*>(x), src, y, 0, w, ws,
-                  static_cast<cudaStream_t>(stream));
+  return ffn_impl(layer, batch, static_cast<const uint16_t*>(x), src, y, 0, w, ws, st);
 }
 
 }  // extern "C"

@@ -197,7 +197,9 @@ int32_t pi_sparse_ffn(const pi_layer* layer, const void* x, int32_t batch,
  *   supported d_model and d_ff.  Larger shapes return PI_ERR_WORKSPACE
  *   with the bytes needed and enqueue nothing.
  * - Set-up: the first call on each device looks up the scratch address; make
- *   it before any stream capture.
+ *   it before any stream capture (a captured first call returns
+ *   PI_ERR_INVALID_ARG).  Every later call outside capture looks the address
+ *   up again, so the scratch stays valid after a device reset.
  * - Concurrency: calls whose kernels may overlap on one device (different
  *   streams, or host threads) race on the shared scratch; serialise them.
  */

@@ -91,6 +91,22 @@ void dequant_q4_0_row(const uint8_t* row, int d, double* out) {
   }
 }
 
+// The value of every 16-bit pattern, decoded once by the functions above, so
+// that widening a row is one table read per element.
+const std::vector<double>& pattern_values(int dtype) {
+  static const std::vector<double> f16 = [] {
+    std::vector<double> t(65536);
+    for (int b = 0; b < 65536; ++b) t[b] = widen_f16_bits((uint16_t)b);
+    return t;
+  }();
+  static const std::vector<double> bf16 = [] {
+    std::vector<double> t(65536);
+    for (int b = 0; b < 65536; ++b) t[b] = widen_bf16_bits((uint16_t)b);
+    return t;
+  }();
+  return dtype == 0 ? f16 : bf16;
+}
+
 // dtype codes: 0 fp16, 1 bf16, 2 Q4_0
 void widen_row(const void* base, int dtype, int64_t row, int d, double* out) {
   if (dtype == 2) {
@@ -98,7 +114,8 @@ void widen_row(const void* base, int dtype, int64_t row, int d, double* out) {
     return;
   }
   const uint16_t* p = static_cast<const uint16_t*>(base) + (size_t)row * d;
-  for (int k = 0; k < d; ++k) out[k] = dtype == 0 ? widen_f16_bits(p[k]) : widen_bf16_bits(p[k]);
+  const double* v = pattern_values(dtype).data();
+  for (int k = 0; k < d; ++k) out[k] = v[p[k]];
 }
 
 // ------------------------------------------------------------ rounding
@@ -187,24 +204,33 @@ void po_rms_cast(const double* x, int32_t B, int32_t d, int32_t adtype, double* 
 void po_predict(const po_layer* L, const double* x, int32_t B, double* a, double* s,
                 uint8_t* mask) {
   const int d = L->d_model, r = L->rank, F = L->d_ff;
-  std::vector<double> w(d > r ? d : r);
+  std::vector<double> w(d > r ? d : r), z(B);
+  // Each token's dot product is summed in index order; the tokens are
+  // interleaved (x and a held index-major) only so that their independent
+  // sums overlap in time.
+  std::vector<double> xt((size_t)d * B), at((size_t)r * B);
+  for (int b = 0; b < B; ++b)
+    for (int k = 0; k < d; ++k) xt[(size_t)k * B + b] = x[(size_t)b * d + k];
   for (int j = 0; j < r; ++j) {
     widen_row(L->w1, L->pdtype, j, d, w.data());
+    for (int b = 0; b < B; ++b) z[b] = 0.0;
+    for (int k = 0; k < d; ++k)
+      for (int b = 0; b < B; ++b) z[b] += w[k] * xt[(size_t)k * B + b];
     for (int b = 0; b < B; ++b) {
-      double z = 0.0;
-      for (int k = 0; k < d; ++k) z += w[k] * x[(size_t)b * d + k];
-      if (L->b1) z += L->b1[j];
-      a[(size_t)b * r + j] = z > 0.0 ? z : 0.0;
+      if (L->b1) z[b] += L->b1[j];
+      a[(size_t)b * r + j] = z[b] > 0.0 ? z[b] : 0.0;
+      at[(size_t)j * B + b] = a[(size_t)b * r + j];
     }
   }
   for (int n = 0; n < F; ++n) {
     widen_row(L->w2, L->pdtype, n, r, w.data());
+    for (int b = 0; b < B; ++b) z[b] = 0.0;
+    for (int j = 0; j < r; ++j)
+      for (int b = 0; b < B; ++b) z[b] += w[j] * at[(size_t)j * B + b];
     for (int b = 0; b < B; ++b) {
-      double z = 0.0;
-      for (int j = 0; j < r; ++j) z += w[j] * a[(size_t)b * r + j];
-      z += L->b2[n];
-      s[(size_t)b * F + n] = z;
-      mask[(size_t)b * F + n] = z > L->threshold ? 1 : 0;
+      z[b] += L->b2[n];
+      s[(size_t)b * F + n] = z[b];
+      mask[(size_t)b * F + n] = z[b] > L->threshold ? 1 : 0;
     }
   }
 }
@@ -234,25 +260,31 @@ void po_band(const double* s, int64_t n, double threshold, double width, uint8_t
 int32_t po_neuron_outputs(const po_layer* L, const double* x, int32_t B, const int64_t* idx,
                           int64_t K, double* h) {
   const int d = L->d_model;
-  std::vector<double> up(d), gate(d);
+  std::vector<double> up(d), gate(d), u(B), g(B), xt((size_t)d * B);
+  for (int b = 0; b < B; ++b)  // x held index-major (see po_predict)
+    for (int c = 0; c < d; ++c) xt[(size_t)c * B + b] = x[(size_t)b * d + c];
   for (int64_t k = 0; k < K; ++k) {
     const int64_t i = idx[k];
     if (i < 0 || i >= L->d_ff) return -1;
     widen_row(L->w_up, L->wdtype, i, d, up.data());
     if (L->act == 1) widen_row(L->w_gate, L->wdtype, i, d, gate.data());
+    // per token, the dot products are summed in index order
+    for (int b = 0; b < B; ++b) u[b] = g[b] = 0.0;
+    for (int c = 0; c < d; ++c)
+      for (int b = 0; b < B; ++b) u[b] += up[c] * xt[(size_t)c * B + b];
+    if (L->act == 1)
+      for (int c = 0; c < d; ++c)
+        for (int b = 0; b < B; ++b) g[b] += gate[c] * xt[(size_t)c * B + b];
     for (int b = 0; b < B; ++b) {
-      const double* xb = x + (size_t)b * d;
-      double u = 0.0;
-      for (int c = 0; c < d; ++c) u += up[c] * xb[c];
       double v;
       if (L->act == 1) {  // ReGLU: relu(gate pre-activation) * up projection
-        double g = 0.0;
-        for (int c = 0; c < d; ++c) g += gate[c] * xb[c];
-        if (L->b_gate) g += L->b_gate[i];
-        v = (g > 0.0 ? g : 0.0) * u;
+        double gb = g[b];
+        if (L->b_gate) gb += L->b_gate[i];
+        v = (gb > 0.0 ? gb : 0.0) * u[b];
       } else {
-        if (L->b_up) u += L->b_up[i];
-        const double rl = u > 0.0 ? u : 0.0;
+        double ub = u[b];
+        if (L->b_up) ub += L->b_up[i];
+        const double rl = ub > 0.0 ? ub : 0.0;
         v = L->act == 2 ? rl * rl : rl;  // Squared-ReLU squares the ReLU output
       }
       h[(size_t)b * K + k] = v;

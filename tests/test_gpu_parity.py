@@ -35,7 +35,10 @@ SMALL = {
         Config(18, "t-q4-sqrelu", 2, 512, 2048, "sqrelu", "q4_0", "f16", 0.015, 1.1, 0.1, 128),
     ]
 }
-BATCHES = [1, 2, 4, 8, 32]
+# every code path by batch: the fused kernels (1, 2, 4), the batched path with
+# B % 4 != 0 (3, 5, 6, 7, 33), the 8-, 16- and 32-token down passes and the
+# 1-, 2-, 4- and 8-tile row GEMMs (8, 12, 16, 24, 32, 48, 64)
+BATCHES = [1, 2, 3, 4, 5, 6, 7, 8, 12, 16, 24, 32, 33, 48, 64]
 
 
 def ftol(cfg):
@@ -262,35 +265,65 @@ def test_layer_pipeline(name, B):
 
 
 # ------------------------------------------------------------------- stack
-def check_stack(layers_or, descs, cfg, x0, B, tol):
+def teacher_forced_stack(layers_or, descs, cfg, x0, B, tol):
+    """Run the GPU stack one layer at a time and check every layer against the
+    oracle fed the GPU's own residual stream (teacher forcing): the layer's
+    index list must match outside the 1e-3 band, and its FFN output must match
+    the oracle's masked FFN on the GPU's own list.  Returns per-layer
+    (K, band neurons where the lists differ, rel-L2)."""
     import activation_sparse_pi_b200 as pi
-    F, nl = cfg.d_ff, len(descs)
+    F = cfg.d_ff
     ws = workspace(descs, B)
     xr = x0.clone().cuda()
-    idx = torch.zeros(nl, F, dtype=torch.int32, device="cuda")
-    cnt = torch.zeros(nl, dtype=torch.int32, device="cuda")
-    pi.pi_ffn_stack(descs, xr, B, idx, cnt, ws)
+    idx = torch.zeros(1, F, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stats = []
+    for l, OL in enumerate(layers_or):
+        x_before = xr.cpu().double().numpy()
+        pi.pi_ffn_stack(pi.layer_array([descs[l]]), xr, B, idx, cnt, ws)
+        torch.cuda.synchronize()
+        x_after = xr.cpu().double().numpy()
+        g = idx[0, : int(cnt.item())].cpu().numpy()
+        xl = oracle.rms_cast(x_before, cfg.adtype)
+        _, s_or, m_or = oracle.predict(OL, xl)
+        diff = check_index_list(g, s_or, OL.threshold, oracle.union_index(m_or))
+        assert np.all(np.diff(g) > 0)
+        y_or = oracle.masked_ffn(OL, xl, g)
+        err = rel_l2(x_after - x_before, y_or)
+        assert err <= tol, (l, err)
+        stats.append((int(g.size), int(diff.size), err))
+    return stats
+
+
+def free_running_drift(layers_or, descs, cfg, x0, B):
+    """End-to-end drift of the whole stack against the oracle's own stack
+    (mask flips near the threshold cascade; reported, not gated)."""
+    import activation_sparse_pi_b200 as pi
+    ws = workspace(descs, B)
+    xr = x0.clone().cuda()
+    pi.pi_ffn_stack(descs, xr, B, None, None, ws)
     torch.cuda.synchronize()
-    out_or, trace = oracle.ffn_stack(layers_or, x0.double().numpy(), cfg.adtype)
-    gi, gc = idx.cpu().numpy(), cnt.cpu().numpy()
-    for l, (I_or, s_or, _) in enumerate(trace):
-        g = gi[l, : gc[l]]
-        diff = check_index_list(g, s_or, layers_or[l].threshold, I_or)
-        if diff.size:
-            return l  # a band decision differs; later layers see other inputs
-    err = rel_l2(xr.cpu().double().numpy(), out_or)
-    assert err <= tol, err
-    return None
+    out_or, _ = oracle.ffn_stack(layers_or, x0.double().numpy(), cfg.adtype)
+    return rel_l2(xr.cpu().double().numpy(), out_or)
 
 
 @pytest.mark.parametrize("name", [n for n in SMALL if SMALL[n].n_layers > 1])
-@pytest.mark.parametrize("B", [1, 2, 8])
+@pytest.mark.parametrize("B", [1, 2, 5, 8, 16])
 def test_stack_parity(name, B):
     cfg = SMALL[name]
     pairs = [small_layer(name, l) for l in range(cfg.n_layers)]
     devs = [device_layer(L) for L, _ in pairs]
     x0 = synth.make_tokens(cfg, B, seed_offset=33)
-    check_stack([OL for _, OL in pairs], [d for _, d in devs], cfg, x0, B, ftol(cfg))
+    ors = [OL for _, OL in pairs]
+    stats = teacher_forced_stack(ors, [d for _, d in devs], cfg, x0, B, ftol(cfg))
+    assert len(stats) == cfg.n_layers
+    drift = free_running_drift(ors, pi_layers(devs), cfg, x0, B)
+    print(f"{name} B={B}: band flips per layer {[s[1] for s in stats]}, drift {drift:.2e}")
+
+
+def pi_layers(devs):
+    import activation_sparse_pi_b200 as pi
+    return pi.layer_array([d for _, d in devs])
 
 
 def test_stack_deterministic():
@@ -308,10 +341,10 @@ def test_stack_deterministic():
 
 
 # ------------------------------------------------- full sizes (sampled)
-FULL_LAYER_CASES = [("opt-6.7b", 1), ("opt-6.7b", 4), ("relu-llama2-13b", 1),
-                    ("relu-llama2-13b", 8), ("falcon-40b", 1), ("falcon-40b", 64),
-                    ("llama2-70b-q4", 1), ("llama2-70b-q4", 8), ("llama2-70b-q4", 32),
-                    ("opt-6.7b-sqrelu", 1)]
+FULL_LAYER_CASES = [("opt-6.7b", 1), ("opt-6.7b", 4), ("opt-6.7b", 16), ("relu-llama2-13b", 1),
+                    ("relu-llama2-13b", 5), ("relu-llama2-13b", 8), ("falcon-40b", 1),
+                    ("falcon-40b", 64), ("llama2-70b-q4", 1), ("llama2-70b-q4", 8),
+                    ("llama2-70b-q4", 32), ("opt-6.7b-sqrelu", 1)]
 
 
 @pytest.mark.slow
@@ -332,14 +365,19 @@ def test_full_size_layer(name, B):
 @pytest.mark.slow
 def test_full_size_opt_stack():
     """The whole 32-layer OPT-6.7B-shaped stack at batch 1 (the benchmarked
-    launch configuration), one token, against the oracle's own stack."""
+    launch configuration), one token, teacher-forced: every layer's index list
+    and output are checked against the oracle."""
     cfg = synth.get_config("opt-6.7b")
     layers = [synth.make_layer(cfg, l, "cuda", "R") for l in range(cfg.n_layers)]
     devs = [device_layer(L) for L in layers]
     x0 = synth.make_tokens(cfg, 1, seed_offset=101)
     ors = [oracle_layer(L) for L in layers]
-    first_flip = check_stack(ors, [d for _, d in devs], cfg, x0, 1, 1e-3)
-    assert first_flip is None or first_flip >= 0
+    stats = teacher_forced_stack(ors, [d for _, d in devs], cfg, x0, 1, 1e-3)
+    assert len(stats) == cfg.n_layers and all(0 < k <= cfg.d_ff for k, _, _ in stats)
+    flips = [(l, s[1]) for l, s in enumerate(stats) if s[1]]
+    drift = free_running_drift(ors, pi_layers(devs), cfg, x0, 1)
+    print(f"opt-6.7b stack: layers with band flips {flips}, max rel-L2 "
+          f"{max(s[2] for s in stats):.2e}, free-running drift {drift:.2e}")
     del layers, devs
     torch.cuda.empty_cache()
 

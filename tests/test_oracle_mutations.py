@@ -18,11 +18,13 @@ from tests import test_oracle_pins as pins
 
 # (name, exact text in pi_oracle.cpp, replacement); each text occurs once
 MUTANTS = [
-    ("predict-no-relu", "a[(size_t)b * r + j] = z > 0.0 ? z : 0.0;", "a[(size_t)b * r + j] = z;"),
-    ("predict-no-b2", "z += L->b2[n];", "(void)0;"),
-    ("predict-no-b1", "if (L->b1) z += L->b1[j];", "(void)0;"),
-    ("predict-tie-active", "z > L->threshold ? 1 : 0", "z >= L->threshold ? 1 : 0"),
-    ("predict-x-transposed", "z += w[k] * x[(size_t)b * d + k];", "z += w[k] * x[(size_t)k * B + b];"),
+    ("predict-no-relu", "a[(size_t)b * r + j] = z[b] > 0.0 ? z[b] : 0.0;",
+     "a[(size_t)b * r + j] = z[b];"),
+    ("predict-no-b2", "z[b] += L->b2[n];", "(void)0;"),
+    ("predict-no-b1", "if (L->b1) z[b] += L->b1[j];", "(void)0;"),
+    ("predict-tie-active", "z[b] > L->threshold ? 1 : 0", "z[b] >= L->threshold ? 1 : 0"),
+    ("predict-x-transposed", "xt[(size_t)k * B + b] = x[(size_t)b * d + k];",
+     "xt[(size_t)k * B + b] = x[(size_t)k * B + b];"),
     ("masked-row-by-position", "widen_row(L->w_down_t, L->wdtype, idx[k], d, row.data());",
      "widen_row(L->w_down_t, L->wdtype, k, d, row.data());"),
     ("masked-h-transposed", "const double hb = h[(size_t)b * K + k];",
@@ -30,9 +32,9 @@ MUTANTS = [
     ("reglu-gate-up-swapped",
      "widen_row(L->w_up, L->wdtype, i, d, up.data());\n    if (L->act == 1) widen_row(L->w_gate, L->wdtype, i, d, gate.data());",
      "widen_row(L->act == 1 ? L->w_gate : L->w_up, L->wdtype, i, d, up.data());\n    if (L->act == 1) widen_row(L->w_up, L->wdtype, i, d, gate.data());"),
-    ("relu-drop-bias", "if (L->b_up) u += L->b_up[i];", "(void)0;"),
-    ("reglu-drop-bias", "if (L->b_gate) g += L->b_gate[i];", "(void)0;"),
-    ("reglu-no-relu", "v = (g > 0.0 ? g : 0.0) * u;", "v = g * u;"),
+    ("relu-drop-bias", "if (L->b_up) ub += L->b_up[i];", "(void)0;"),
+    ("reglu-drop-bias", "if (L->b_gate) gb += L->b_gate[i];", "(void)0;"),
+    ("reglu-no-relu", "v = (gb > 0.0 ? gb : 0.0) * u[b];", "v = gb * u[b];"),
     ("sqrelu-unsquared", "v = L->act == 2 ? rl * rl : rl;", "v = rl;"),
     ("q4-nibbles-swapped", "const int lo = p[2 + j] & 0x0f;\n      const int hi = p[2 + j] >> 4;",
      "const int hi = p[2 + j] & 0x0f;\n      const int lo = p[2 + j] >> 4;"),
@@ -48,8 +50,8 @@ MUTANTS = [
     ("round-ties-away", "std::nearbyint(std::ldexp(ax, -qe))", "std::round(std::ldexp(ax, -qe))"),
     ("bf16-exponent-shift-8", "std::ldexp((double)(128 + m), e - 134)",
      "std::ldexp((double)(128 + m), e - 126)"),
-    ("bf16-read-as-f16", "out[k] = dtype == 0 ? widen_f16_bits(p[k]) : widen_bf16_bits(p[k]);",
-     "out[k] = widen_f16_bits(p[k]);"),
+    ("bf16-read-as-f16", "const double* v = pattern_values(dtype).data();",
+     "const double* v = pattern_values(0).data();"),
     ("bf16-fraction-7-as-8", "const int m = b & 0x7f;\n  double v;\n  if (e == 0) {\n    v = std::ldexp((double)m, -133);",
      "const int m = b & 0xff;\n  double v;\n  if (e == 0) {\n    v = std::ldexp((double)m, -133);"),
     ("f16-subnormal-scale", "v = std::ldexp((double)m, -24);", "v = std::ldexp((double)m, -25);"),

@@ -3,16 +3,18 @@
 It must give what pi_sparse_ffn gives on the same inputs (within the FFN
 tolerance of the parity tests, and in fact bit for bit, since both run the
 same kernels in the same order), on calls made back to back so that the second
-finds the scratch dirty from the first.  This file stands alone (run it by
-itself or after the rest of the suite) and is collected last.
+finds the scratch dirty from the first; and both must match the fp64 oracle's
+masked FFN on the same neuron list.  This file stands alone (run it by itself
+or after the rest of the suite) and is collected last.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from synth.configs import Config
-from tests._util import device_layer, rel_l2, to16
+from tests._util import device_layer, oracle_layer, rel_l2, to16
 
 pytestmark = pytest.mark.gpu
 
@@ -42,14 +44,17 @@ def _lib():
 def _inputs(cfg, B, seed):
     L = synth.make_layer(cfg, 0, "cpu", "R")
     Ld, desc = device_layer(L)
-    x = to16(synth.make_tokens(cfg, B, seed_offset=seed), cfg.adtype).cuda()
+    xf = synth.make_tokens(cfg, B, seed_offset=seed)
+    x = to16(xf, cfg.adtype).cuda()
     rng = np.random.default_rng(cfg.d_ff * 7 + B)
     n = max(1, cfg.d_ff // 5)
     I = rng.permutation(cfg.d_ff)[:n].astype(np.int32)
     idx = torch.zeros(cfg.d_ff, dtype=torch.int32, device="cuda")
     idx[:n] = torch.from_numpy(I).cuda()
     cnt = torch.tensor([n], dtype=torch.int32, device="cuda")
-    return Ld, desc, x, idx, cnt
+    # what the oracle says these inputs give
+    expect = oracle.masked_ffn(oracle_layer(L), xf.double().numpy(), I)
+    return (Ld, expect), desc, x, idx, cnt
 
 
 def _reference(desc, x, B, idx, cnt, d):
@@ -73,8 +78,9 @@ def test_static_scratch_matches_workspace_call(name):
     cfg, batches = CASES[name]
     tol = 2e-3 if cfg.wdtype == "q4_0" else 1e-3
     for B in batches:
-        keep, desc, x, idx, cnt = _inputs(cfg, B, seed=B)
+        (keep, expect), desc, x, idx, cnt = _inputs(cfg, B, seed=B)
         want = _reference(desc, x, B, idx, cnt, cfg.d_model)
+        assert rel_l2(want, expect) <= tol, (B, rel_l2(want, expect))
         # two calls in a row on one stream, no synchronisation between them
         y1 = _static(desc, x, B, idx, cnt, cfg.d_model)
         y2 = _static(desc, x, B, idx, cnt, cfg.d_model)
@@ -82,6 +88,7 @@ def test_static_scratch_matches_workspace_call(name):
         for y in (y1, y2):
             got = y.cpu().double().numpy()
             assert np.isfinite(got).all()
+            assert rel_l2(got, expect) <= tol, (B, rel_l2(got, expect))
             assert rel_l2(got, want) <= tol, (B, rel_l2(got, want))
             assert np.array_equal(got, want), f"batch {B}: not bit-identical to pi_sparse_ffn"
 
@@ -91,8 +98,8 @@ def test_static_scratch_reused_across_shapes():
     # after it must not see them
     big_cfg, _ = CASES["relu-f16-8192"]
     small_cfg, _ = CASES["toy"]
-    kb, db, xb, ib, cb = _inputs(big_cfg, 4, seed=1)
-    ks, ds, xs, is_, cs = _inputs(small_cfg, 2, seed=2)
+    (kb, eb), db, xb, ib, cb = _inputs(big_cfg, 4, seed=1)
+    (ks, es), ds, xs, is_, cs = _inputs(small_cfg, 2, seed=2)
     want_b = _reference(db, xb, 4, ib, cb, big_cfg.d_model)
     want_s = _reference(ds, xs, 2, is_, cs, small_cfg.d_model)
     outs = []
@@ -102,4 +109,6 @@ def test_static_scratch_reused_across_shapes():
     torch.cuda.synchronize()
     for which, y in outs:
         want = want_b if which == "b" else want_s
-        assert np.array_equal(y.cpu().double().numpy(), want), which
+        got = y.cpu().double().numpy()
+        assert np.array_equal(got, want), which
+        assert rel_l2(got, eb if which == "b" else es) <= 1e-3, which
