@@ -8,7 +8,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpi.so")
 SOURCES = ["pi_api.cu"]
-HEADERS = ["pi_common.cuh", "pi_predict.cuh", "pi_ffn.cuh", "pi_generic.cuh"]
+HEADERS = ["pi_common.cuh", "pi_predict.cuh", "pi_ffn.cuh", "pi_generic.cuh", "pi_umma.cuh"]
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",
     "-gencode", "arch=compute_100a,code=sm_100a",
