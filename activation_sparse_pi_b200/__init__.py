@@ -26,6 +26,7 @@ from .binding import (  # noqa: F401
     pi_ffn_stack_timed,
     pi_last_error,
     pi_launch_count,
+    pi_permute_layer,
     pi_predict,
     pi_sparse_ffn,
     pi_sparse_ffn_static,

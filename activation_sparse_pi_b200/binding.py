@@ -22,7 +22,7 @@ ACTS = {"relu": PI_RELU, "reglu": PI_REGLU, "sqrelu": PI_SQRELU}
 EXPORTS = (
     "pi_status_string", "pi_last_error", "pi_device_error", "pi_launch_count", "pi_workspace_size",
     "pi_predict", "pi_compact", "pi_sparse_ffn", "pi_ffn_stack", "pi_ffn_stack_timed",
-    "pi_sparse_ffn_static",
+    "pi_sparse_ffn_static", "pi_permute_layer",
 )
 
 
@@ -90,6 +90,9 @@ def lib():
         L.pi_ffn_stack_timed.argtypes = [ctypes.POINTER(PiLayer), c_int32, c_void_p, c_int32,
                                          c_void_p, c_void_p, c_void_p, c_size_t, c_void_p,
                                          ctypes.POINTER(c_void_p)]
+        L.pi_permute_layer.restype = c_int32
+        L.pi_permute_layer.argtypes = [ctypes.POINTER(PiLayer), c_void_p, ctypes.POINTER(PiLayer),
+                                       c_void_p]
         _lib = L
     return _lib
 
@@ -217,3 +220,9 @@ def pi_ffn_stack_timed(layers, x_resid, batch, idx_out, count_out, workspace, ff
     _check(lib().pi_ffn_stack_timed(arr, len(arr), _ptr(x_resid), int(batch), _ptr(idx_out),
                                     _ptr(count_out), _ptr(workspace), _nbytes(workspace),
                                     _stream(stream), ev), "pi_ffn_stack_timed")
+
+
+def pi_permute_layer(src, perm, dst, stream=None):
+    """src, dst: PiLayer descriptors; perm: int32 device tensor [d_ff]."""
+    _check(lib().pi_permute_layer(ctypes.byref(src), _ptr(perm), ctypes.byref(dst),
+                                  _stream(stream)), "pi_permute_layer")

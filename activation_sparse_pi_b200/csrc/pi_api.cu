@@ -679,8 +679,7 @@ bool make_tmap16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows
 }
 
 bool umma_ok(const pi_layer* L, int B) {
-  return (L->wdtype == PI_F16 || L->wdtype == PI_BF16) && B >= kUmmaMinBatch && B <= 64 &&
-         L->d_model % kUmmaM == 0 && tmap_encoder() != nullptr;
+  return B >= kUmmaMinBatch && B <= 64 && L->d_model % kUmmaM == 0 && tmap_encoder() != nullptr;
 }
 
 // pipeline stages that fit two CTAs per SM (at least 2, at most 6)
@@ -690,37 +689,37 @@ constexpr int umma_ns(int stage_bytes) {
 }
 
 template <int DT, int ACT, int N>
-cudaError_t launch_umma_up_n(const pi_layer* L, const CUtensorMap& ta, const CUtensorMap& ta2,
-                             const CUtensorMap& tx, const UmmaParams& p, cudaStream_t st) {
+cudaError_t launch_umma_up_n(const pi_layer* L, const CUtensorMap& tx, const UmmaParams& p,
+                             cudaStream_t st) {
   constexpr int NMAT = ACT == 1 ? 2 : 1;
   constexpr int STAGE = umma_up_stage<NMAT, N>();
   constexpr int NS = umma_ns(STAGE);
   const int tiles = (L->d_ff + kUmmaM - 1) / kUmmaM;
   return launch(k_umma_up<DT, ACT, N, NS>, dim3(tiles), dim3(kUmmaThreads),
-                (size_t)NS * STAGE + 1024, st, ta, ta2, tx, p);
+                (size_t)NS * STAGE + 1024, st, tx, p);
 }
 
 template <int DT, int N>
-cudaError_t launch_umma_down_n(const pi_layer* L, int S, const CUtensorMap& tw,
-                               const CUtensorMap& th, const CUtensorMap& tl, const UmmaParams& p,
-                               cudaStream_t st) {
+cudaError_t launch_umma_down_n(const pi_layer* L, int S, const CUtensorMap& th,
+                               const CUtensorMap& tl, const UmmaParams& p, cudaStream_t st) {
   constexpr int STAGE = umma_down_stage<N>();
   constexpr int NS = umma_ns(STAGE);
   return launch(k_umma_down<DT, N, NS>, dim3(L->d_model / kUmmaM, S), dim3(kUmmaThreads),
-                (size_t)NS * STAGE + 1024, st, tw, th, tl, p);
+                (size_t)NS * STAGE + 1024, st, th, tl, p);
 }
 
 template <int DT, int ACT>
-cudaError_t umma_up_act(const pi_layer* L, int N, const CUtensorMap& ta, const CUtensorMap& ta2,
-                        const CUtensorMap& tx, const UmmaParams& p, cudaStream_t st) {
+cudaError_t umma_up_act(const pi_layer* L, int N, const CUtensorMap& tx, const UmmaParams& p,
+                        cudaStream_t st) {
   switch (N) {
-    case 16: return launch_umma_up_n<DT, ACT, 16>(L, ta, ta2, tx, p, st);
-    case 32: return launch_umma_up_n<DT, ACT, 32>(L, ta, ta2, tx, p, st);
-    case 48: return launch_umma_up_n<DT, ACT, 48>(L, ta, ta2, tx, p, st);
-    default: return launch_umma_up_n<DT, ACT, 64>(L, ta, ta2, tx, p, st);
+    case 16: return launch_umma_up_n<DT, ACT, 16>(L, tx, p, st);
+    case 32: return launch_umma_up_n<DT, ACT, 32>(L, tx, p, st);
+    case 48: return launch_umma_up_n<DT, ACT, 48>(L, tx, p, st);
+    default: return launch_umma_up_n<DT, ACT, 64>(L, tx, p, st);
   }
 }
 
+// DT: 0 fp16, 1 bf16, 2 Q4_0 weights (pi_umma.cuh).
 template <int DT>
 cudaError_t umma_ffn(const pi_layer* L, int B, const uint16_t* x, const int32_t* idx,
                      const int32_t* count, uint16_t* hh, uint16_t* hl, float* part, int S,
@@ -728,18 +727,18 @@ cudaError_t umma_ffn(const pi_layer* L, int B, const uint16_t* x, const int32_t*
   const int d = L->d_model, F = L->d_ff;
   const int N = (B + 15) / 16 * 16;
   const bool reglu = L->act == PI_REGLU;
-  CUtensorMap ta, ta2, tx, tw, th, tl;
-  const uint64_t rb = (uint64_t)d * 2;
-  if (!make_tmap16(&ta, reglu ? L->w_gate : L->w_up, d, F, rb, kUmmaK, 1) ||
-      !make_tmap16(&ta2, L->w_up, d, F, rb, kUmmaK, 1) ||
-      !make_tmap16(&tx, x, d, B, rb, kUmmaK, N) ||
-      !make_tmap16(&tw, L->w_down_t, d, F, rb, kUmmaK, 1) ||
+  CUtensorMap tx{}, th{}, tl{};
+  if (!make_tmap16(&tx, x, d, B, (uint64_t)d * 2, kUmmaK, N) ||
       !make_tmap16(&th, hh, F, B, (uint64_t)F * 2, kUmmaK, N) ||
       !make_tmap16(&tl, hl, F, B, (uint64_t)F * 2, kUmmaK, N))
     return cudaErrorInvalidValue;
   UmmaParams p{};
   p.idx = idx;
   p.count = count;
+  p.wa = static_cast<const uint8_t*>(reglu ? L->w_gate : L->w_up);
+  p.wa2 = static_cast<const uint8_t*>(L->w_up);
+  p.wd = static_cast<const uint8_t*>(L->w_down_t);
+  p.rb = (uint32_t)ffn_row_bytes(L);
   p.bias = reglu ? L->b_gate : L->b_up;
   p.hh = hh;
   p.hl = hl;
@@ -747,15 +746,15 @@ cudaError_t umma_ffn(const pi_layer* L, int B, const uint16_t* x, const int32_t*
   p.d = d;
   p.F = F;
   p.B = B;
-  cudaError_t e = L->act == PI_REGLU ? umma_up_act<DT, 1>(L, N, ta, ta2, tx, p, st)
-                : L->act == PI_SQRELU ? umma_up_act<DT, 2>(L, N, ta, ta2, tx, p, st)
-                                      : umma_up_act<DT, 0>(L, N, ta, ta2, tx, p, st);
+  cudaError_t e = L->act == PI_REGLU ? umma_up_act<DT, 1>(L, N, tx, p, st)
+                : L->act == PI_SQRELU ? umma_up_act<DT, 2>(L, N, tx, p, st)
+                                      : umma_up_act<DT, 0>(L, N, tx, p, st);
   if (e != cudaSuccess) return e;
   switch (N) {
-    case 16: return launch_umma_down_n<DT, 16>(L, S, tw, th, tl, p, st);
-    case 32: return launch_umma_down_n<DT, 32>(L, S, tw, th, tl, p, st);
-    case 48: return launch_umma_down_n<DT, 48>(L, S, tw, th, tl, p, st);
-    default: return launch_umma_down_n<DT, 64>(L, S, tw, th, tl, p, st);
+    case 16: return launch_umma_down_n<DT, 16>(L, S, th, tl, p, st);
+    case 32: return launch_umma_down_n<DT, 32>(L, S, th, tl, p, st);
+    case 48: return launch_umma_down_n<DT, 48>(L, S, th, tl, p, st);
+    default: return launch_umma_down_n<DT, 64>(L, S, th, tl, p, st);
   }
 }
 
@@ -815,9 +814,9 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     uint16_t* hl = hh + (size_t)L->d_ff * B;
     G = umma_slices(d, B, num_sms());
     const cudaError_t e =
-        L->wdtype == PI_BF16
-            ? umma_ffn<1>(L, B, x, src.idx, src.count, hh, hl, part, G, st)
-            : umma_ffn<0>(L, B, x, src.idx, src.count, hh, hl, part, G, st);
+        L->wdtype == PI_BF16  ? umma_ffn<1>(L, B, x, src.idx, src.count, hh, hl, part, G, st)
+        : L->wdtype == PI_Q4_0 ? umma_ffn<2>(L, B, x, src.idx, src.count, hh, hl, part, G, st)
+                               : umma_ffn<0>(L, B, x, src.idx, src.count, hh, hl, part, G, st);
     if (e != cudaSuccess)
       return fail(PI_ERR_CUDA, "tensor-core FFN launch failed: %s", cudaGetErrorString(e));
   } else {
@@ -872,6 +871,29 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
   if (mode == 0) PI_CUDA((launch(k_reduce<0>, rg, rt, 0, st, (const float*)part, G, n4, out)));
   else PI_CUDA((launch(k_reduce<1>, rg, rt, 0, st, (const float*)part, G, n4, out)));
   return PI_OK;
+}
+
+// One neuron-indexed tensor of a layer permuted into dst (see pi_permute_layer).
+cudaError_t gather_rows(const void* src, void* dst, const int32_t* perm, int n, size_t row_bytes,
+                        cudaStream_t st) {
+  const int nsm = num_sms();
+  if (row_bytes % 16 == 0) {
+    const int units = (int)(row_bytes / 16);
+    const long long total = (long long)n * units;
+    const int blocks = (int)std::min<long long>((total + 255) / 256, 8ll * nsm);
+    return launch(k_gather_rows<16>, dim3(blocks), dim3(256), 0, st,
+                  static_cast<const uint8_t*>(src), static_cast<uint8_t*>(dst), perm, n, units);
+  }
+  const int units = (int)(row_bytes / 4);
+  const long long total = (long long)n * units;
+  const int blocks = (int)std::min<long long>((total + 255) / 256, 8ll * nsm);
+  return launch(k_gather_rows<4>, dim3(blocks), dim3(256), 0, st,
+                static_cast<const uint8_t*>(src), static_cast<uint8_t*>(dst), perm, n, units);
+}
+
+bool overlaps(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + bytes && y < x + bytes;
 }
 
 }  // namespace
@@ -1089,6 +1111,42 @@ int32_t pi_sparse_ffn_static(const pi_layer* layer, const void* x, int32_t batch
   }
   FfnSrc src{idx, count, nullptr, 0, nullptr, nullptr};
   return ffn_impl(layer, batch, static_cast<const uint16_t*>(x), src, y, 0, w, ws, st);
+}
+
+// Hot-row ordering: the layer with its neurons renumbered (dst neuron i =
+// src neuron perm[i]).  Every neuron-indexed tensor is gathered row by row
+// into the caller's dst buffers; W1, b1 and the threshold are not touched.
+int32_t pi_permute_layer(const pi_layer* src, const int32_t* perm, const pi_layer* dst,
+                         void* stream) {
+  if (int32_t s = validate_layer(src)) return s;
+  if (int32_t s = validate_layer(dst)) return s;
+  if (!perm || !aligned16(perm)) return fail(PI_ERR_INVALID_ARG, "perm must be a 16-byte aligned device pointer");
+  if (src->d_model != dst->d_model || src->d_ff != dst->d_ff || src->wdtype != dst->wdtype ||
+      src->adtype != dst->adtype || src->act != dst->act || src->pred.rank != dst->pred.rank)
+    return fail(PI_ERR_INVALID_ARG, "src and dst must have the same shapes, dtypes and activation");
+  if ((src->b_up == nullptr) != (dst->b_up == nullptr) ||
+      (src->b_gate == nullptr) != (dst->b_gate == nullptr))
+    return fail(PI_ERR_INVALID_ARG, "src and dst must both have, or both lack, each bias");
+  const int F = src->d_ff;
+  const size_t rb = ffn_row_bytes(src);
+  const size_t rb2 = (size_t)src->pred.rank * 2;
+  struct T { const void* s; void* d; size_t row; };
+  const T ts[] = {
+      {src->w_up, const_cast<void*>(dst->w_up), rb},
+      {src->w_gate, const_cast<void*>(dst->w_gate), rb},
+      {src->w_down_t, const_cast<void*>(dst->w_down_t), rb},
+      {src->pred.w2, const_cast<void*>(dst->pred.w2), rb2},
+      {src->pred.b2, const_cast<float*>(dst->pred.b2), 4},
+      {src->b_up, const_cast<float*>(dst->b_up), 4},
+      {src->b_gate, const_cast<float*>(dst->b_gate), 4},
+  };
+  for (const T& t : ts)
+    if (t.s && (t.d == t.s || overlaps(t.s, t.d, t.row * F)))
+      return fail(PI_ERR_INVALID_ARG, "a permuted dst tensor overlaps its src tensor");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (const T& t : ts)
+    if (t.s) PI_CUDA(gather_rows(t.s, t.d, perm, F, t.row, st));
+  return PI_OK;
 }
 
 }  // extern "C"

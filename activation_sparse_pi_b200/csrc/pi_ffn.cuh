@@ -709,6 +709,37 @@ __global__ void __launch_bounds__(kQ4Threads, B == 1 ? 2 : 1) k_ffn_q4(FfnParams
   }
 }
 
+// ------------------------------------------------------ row permutation
+// dst row i = src row perm[i] (rows of row_bytes bytes, V-byte units: 16 when
+// row_bytes % 16 == 0, else 4).  Grid-stride over (row, unit) pairs, so
+// consecutive threads copy consecutive units of one row.  Ids outside
+// [0, n) are flagged and their destination rows left untouched.
+template <int V>
+__global__ void __launch_bounds__(256) k_gather_rows(const uint8_t* __restrict__ src,
+                                                     uint8_t* __restrict__ dst,
+                                                     const int32_t* __restrict__ perm, int n,
+                                                     int row_units) {
+  pdl_wait();
+  pdl_trigger();
+  const long long total = (long long)n * row_units;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(e / row_units), u = (int)(e % row_units);
+    const int j = perm[i];
+    if (j < 0 || j >= n) {
+      if (u == 0) set_error(kErrBadIndex);
+      continue;
+    }
+    if constexpr (V == 16) {
+      reinterpret_cast<uint4*>(dst)[e] =
+          ldg_stream(src + ((size_t)j * row_units + u) * 16);
+    } else {
+      reinterpret_cast<uint32_t*>(dst)[e] =
+          reinterpret_cast<const uint32_t*>(src)[(size_t)j * row_units + u];
+    }
+  }
+}
+
 // ------------------------------------------------------ partial reduction
 // out[i] = sum over g = 0..G-1 of part[g][i], MODE 0 writes y, MODE 1 adds into
 // the residual stream.  n4 = number of float4 columns (B*d/4).  A CTA covers 8

@@ -8,14 +8,18 @@
 //   up:   H[k][n]  = act(W_act[idx_k] . x_n (+ b), W_up[idx_k] . x_n)
 //   down: y[n][c]  = sum_k H[k][n] W_down^T[idx_k][c]
 // Both run here as tcgen05.mma (kind::f16, fp32 accumulation in tensor
-// memory) on operands that the tensor memory accelerator gathers straight
-// from HBM into 128-byte-swizzled shared memory:
-//   - weight rows: cp.async.bulk.tensor .tile::gather4 (four neuron ids per
-//     instruction, 64 elements = 128 bytes of each row);
-//   - tokens (up) and H (down): ordinary 2-D tensor tiles, rows past the batch
-//     filled with zeros by the copy engine.
-// One thread issues the copies, one thread the MMAs; four warps read the
-// accumulator out of tensor memory (tcgen05.ld) for the epilogue.
+// memory) on operands staged in 128-byte-swizzled shared memory:
+//   - weight rows: four warps gather the listed rows with coalesced 128-bit
+//     loads (eight threads per 128-byte piece of a row) and store them in
+//     the swizzled layout, dequantizing Q4_0 blocks on the way.  (A first
+//     version gathered them with cp.async.bulk.tensor .tile::gather4; at 128
+//     bytes per row and four rows per instruction the copy engine delivered
+//     about 1.7 TB/s, a quarter of what plain loads reach.)
+//   - tokens (up) and H (down): 2-D tensor tiles copied by the tensor memory
+//     accelerator, rows past the batch filled with zeros by the copy engine.
+// One thread issues the copies, one thread the MMAs; the four builder warps
+// then read the accumulator out of tensor memory (tcgen05.ld) for the
+// epilogue.
 //
 // Precision: the products of 16-bit operands are exact and accumulate in
 // fp32.  H is the one intermediate that must be rounded to a 16-bit MMA
@@ -105,16 +109,6 @@ __host__ __device__ constexpr uint32_t idesc_f16() {
 }
 
 // ---------------------------------------------------------------- TMA
-// Four rows (r0..r3) of a 2-D tensor, box {64 elements, 1 row}, into 512
-// contiguous bytes of shared memory; completion counted on *bar.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* tm, int col, int r0,
-                                            int r1, int r2, int r3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(tm), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
-      : "memory");
-}
 // One box of a 2-D tensor at (c0 = inner coordinate, c1 = row).
 __device__ __forceinline__ void tma_load2d(void* dst, const CUtensorMap* tm, int c0, int c1,
                                            uint64_t* bar) {
@@ -125,6 +119,75 @@ __device__ __forceinline__ void tma_load2d(void* dst, const CUtensorMap* tm, int
       : "memory");
 }
 
+// ---------------------------------------------------------------- Q4_0
+// The copy engine cannot dequantize, so with Q4_0 weights (DT 2) four warps
+// build the weight operand themselves: each thread loads two consecutive
+// blocks of a row (36 bytes, 4-byte aligned, as nine 32-bit words), turns
+// them into 64 fp16 values (q - 8) * scale -- exact (q - 8) from the
+// exponent trick 0x6400 | q = 1024 + q, then one rounding in the multiply by
+// the block scale -- and stores them as eight 16-byte chunks in the swizzled
+// layout.  The tensor cores then multiply fp16 x fp16 exactly with fp32
+// accumulation; the one rounding of each weight (relative 2^-12 at most)
+// keeps the FFN far inside its 2e-3 tolerance.
+__device__ __forceinline__ void ld_q4_pair(const uint8_t* p, uint32_t (&w)[9]) {
+  const uint32_t* q = reinterpret_cast<const uint32_t*>(p);
+#pragma unroll
+  for (int k = 0; k < 9; ++k) w[k] = __ldg(q + k);
+}
+
+// Two fp16 values (q - 8) * scale for the nibbles q held in two bytes of v
+// (each byte 0..15; sel picks them: 0x4140 bytes 0-1, 0x4342 bytes 2-3).
+// Bits and half2 values are converted with intrinsics, not pointer casts.
+__device__ __forceinline__ uint32_t q4_h2(uint32_t v, uint32_t sel, __half2 scale2) {
+  const uint32_t biased = __byte_perm(v, 0x64646464u, sel);  // halves 0x6400 | q = 1024 + q
+  const __half2 qb = __halves2half2(__ushort_as_half((unsigned short)(biased & 0xffffu)),
+                                    __ushort_as_half((unsigned short)(biased >> 16)));
+  const __half2 r = __hmul2(__hsub2(qb, __float2half2_rn(1032.f)), scale2);
+  return (uint32_t)__half_as_ushort(__low2half(r)) |
+         ((uint32_t)__half_as_ushort(__high2half(r)) << 16);
+}
+
+// 36 bytes = blocks A and B -> chunks c = 0..7 of 8 consecutive values each
+// (chunks 0-3 from block A, 4-7 from block B; within a block chunk 0 is the
+// low nibbles of bytes 0-7, chunk 1 of bytes 8-15, chunks 2-3 the high ones).
+__device__ __forceinline__ void dq_q4_pair(const uint32_t (&w)[9], uint4 (&out)[8]) {
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    uint32_t nb[4];
+    uint32_t sbits;
+    if (b == 0) {
+      sbits = w[0] & 0xffffu;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) nb[k] = __funnelshift_r(w[k], w[k + 1], 16);
+    } else {
+      sbits = w[4] >> 16;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) nb[k] = w[5 + k];
+    }
+    const __half s = __ushort_as_half((unsigned short)sbits);
+    const __half2 s2 = __halves2half2(s, s);
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      lo[k] = nb[k] & 0x0F0F0F0Fu;
+      hi[k] = (nb[k] >> 4) & 0x0F0F0F0Fu;
+    }
+    out[4 * b + 0] = make_uint4(q4_h2(lo[0], 0x4140u, s2), q4_h2(lo[0], 0x4342u, s2),
+                                q4_h2(lo[1], 0x4140u, s2), q4_h2(lo[1], 0x4342u, s2));
+    out[4 * b + 1] = make_uint4(q4_h2(lo[2], 0x4140u, s2), q4_h2(lo[2], 0x4342u, s2),
+                                q4_h2(lo[3], 0x4140u, s2), q4_h2(lo[3], 0x4342u, s2));
+    out[4 * b + 2] = make_uint4(q4_h2(hi[0], 0x4140u, s2), q4_h2(hi[0], 0x4342u, s2),
+                                q4_h2(hi[1], 0x4140u, s2), q4_h2(hi[1], 0x4342u, s2));
+    out[4 * b + 3] = make_uint4(q4_h2(hi[2], 0x4140u, s2), q4_h2(hi[2], 0x4342u, s2),
+                                q4_h2(hi[3], 0x4140u, s2), q4_h2(hi[3], 0x4342u, s2));
+  }
+}
+
+// Stages of raw Q4_0 blocks the operand builders keep in flight in registers
+// (per thread: NMAT x 36 bytes per stage).
+template <int NMAT>
+__host__ __device__ constexpr int q4_ahead() { return NMAT == 1 ? 4 : 2; }
+
 // ---------------------------------------------------------------- kernels
 constexpr int kUmmaThreads = 192;  // warp 0 copies, warp 1 MMAs, warps 2-5 epilogue
 constexpr int kUmmaM = 128;        // neuron rows (up) / output columns (down) per tile
@@ -133,6 +196,10 @@ constexpr int kUmmaK = 64;         // contraction elements per stage (one 128-by
 struct UmmaParams {
   const int32_t* idx;      // neuron list (first *count entries)
   const int32_t* count;
+  const uint8_t* wa;       // Q4_0 rows (DT 2): activation rows (W_up or W_gate) ...
+  const uint8_t* wa2;      // ... W_up rows (ReGLU) ...
+  const uint8_t* wd;       // ... and W_down^T rows
+  uint32_t rb;             // bytes of one Q4_0 row
   const float* bias;       // up: b_up (ReLU, Squared-ReLU) or b_gate (ReGLU), or null
   uint16_t* hh;            // [B x F] 16-bit hi part of H (token-major)
   uint16_t* hl;            // [B x F] 16-bit lo part
@@ -159,20 +226,31 @@ __device__ __forceinline__ float from16(uint16_t u) {
   else return __uint_as_float((uint32_t)u << 16);
 }
 
+// Stages of 16-bit weight chunks the builders keep in flight in registers.
+template <int NMAT>
+__host__ __device__ constexpr int umma_ahead16() { return NMAT == 1 ? 2 : 1; }
+
 // Gathered up projection + activation.  One CTA per tile of 128 listed
 // neurons (tiles past the device-side count exit at once); the contraction
-// runs over d in stages of 64.  DT: 0 fp16, 1 bf16 weights and tokens.
-// ACT: 0 ReLU, 1 ReGLU (gate rows in tm_a, up rows in tm_a2), 2 Squared-ReLU.
-// N: tokens per MMA (the batch rounded up to a multiple of 16).
+// runs over d in stages of 64.  DT: 0 fp16, 1 bf16 (weights and tokens),
+// 2 Q4_0 weights with fp16 tokens.  ACT: 0 ReLU, 1 ReGLU (gate rows in p.wa,
+// up rows in p.wa2), 2 Squared-ReLU.  N: tokens per MMA (the batch rounded up
+// to a multiple of 16).
+//   warp 0     copies the stage's token tile (TMA, rows past the batch zero)
+//   warp 1     issues the MMAs (one thread) and owns the tensor memory
+//   warps 2-5  build the weight operand: the tile's 128 gathered rows, 64
+//              elements per stage, with 128-bit loads (8 threads per row, so
+//              a warp instruction reads four whole 128-byte row pieces) stored
+//              in the swizzled layout; then the epilogue
 template <int DT, int ACT, int N, int NS>
 __global__ void __launch_bounds__(kUmmaThreads, 1)
-    k_umma_up(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a2,
-              const __grid_constant__ CUtensorMap tm_x, UmmaParams p) {
+    k_umma_up(const __grid_constant__ CUtensorMap tm_x, UmmaParams p) {
   constexpr int NMAT = ACT == 1 ? 2 : 1;
+  constexpr bool Q4 = DT == 2;
   constexpr int ABYTES = kUmmaM * kUmmaK * 2;  // 16 KB per matrix
   constexpr int STAGE = umma_up_stage<NMAT, N>();
   constexpr uint32_t NCOL = NMAT * N <= 32 ? 32 : NMAT * N <= 64 ? 64 : NMAT * N <= 128 ? 128 : 256;
-  constexpr uint32_t IDESC = idesc_f16<DT, kUmmaM, N, 0, 0>();
+  constexpr uint32_t IDESC = idesc_f16<Q4 ? 0 : DT, kUmmaM, N, 0, 0>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -200,7 +278,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   }
   if (t == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + kUmmaM);  // the token copy + 128 builder threads
       mbar_init(&empty[s], 1);
     }
     mbar_init(&done, 1);
@@ -214,21 +292,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   const int nst = p.d / kUmmaK;
 
   if (warp == 0) {
-    if (lane == 0) {  // copy engine feeder
+    if (lane == 0) {  // token tiles
       for (int i = 0; i < nst; ++i) {
         const int s = i % NS;
         if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) break;
-        uint8_t* st = smem + (size_t)s * STAGE;
-        mbar_arrive_expect_tx(&full[s], STAGE);
-#pragma unroll 1
-        for (int q = 0; q < kUmmaM / 4; ++q) {
-          const int r0 = max(ids[4 * q], 0), r1 = max(ids[4 * q + 1], 0);
-          const int r2 = max(ids[4 * q + 2], 0), r3 = max(ids[4 * q + 3], 0);
-          tma_gather4(st + 512 * q, &tm_a, i * kUmmaK, r0, r1, r2, r3, &full[s]);
-          if constexpr (NMAT == 2)
-            tma_gather4(st + ABYTES + 512 * q, &tm_a2, i * kUmmaK, r0, r1, r2, r3, &full[s]);
-        }
-        tma_load2d(st + NMAT * ABYTES, &tm_x, i * kUmmaK, 0, &full[s]);
+        mbar_arrive_expect_tx(&full[s], N * kUmmaK * 2);
+        tma_load2d(smem + (size_t)s * STAGE + NMAT * ABYTES, &tm_x, i * kUmmaK, 0, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -253,14 +322,104 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     }
     __syncwarp();
   } else {
+    const int m = t - 64;  // 0..127
+    bool ok = true;
+    if constexpr (Q4) {
+      // thread m builds row m: two Q4_0 blocks (36 bytes) per stage
+      const int id = max(ids[m], 0);
+      const uint8_t* rowp[NMAT];
+      rowp[0] = p.wa + (size_t)id * p.rb;
+      if constexpr (NMAT == 2) rowp[NMAT - 1] = p.wa2 + (size_t)id * p.rb;
+      constexpr int QA = q4_ahead<NMAT>();
+      uint32_t raw[QA][NMAT][9];
+#pragma unroll
+      for (int j = 0; j < QA; ++j)
+        if (j < nst)
+#pragma unroll
+          for (int mm = 0; mm < NMAT; ++mm) ld_q4_pair(rowp[mm] + 36 * j, raw[j][mm]);
+      const uint32_t rsw = (uint32_t)(m & 7);
+      for (int i0 = 0; i0 < nst && ok; i0 += QA) {
+#pragma unroll
+        for (int j = 0; j < QA; ++j) {
+          const int i = i0 + j;
+          if (i < nst && ok) {
+            const int s = i % NS;
+            if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
+            if (ok) {
+              uint8_t* row0 = smem + (size_t)s * STAGE + (m >> 3) * 1024 + (m & 7) * 128;
+#pragma unroll
+              for (int mm = 0; mm < NMAT; ++mm) {
+                uint4 ch[8];
+                dq_q4_pair(raw[j][mm], ch);
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                  *reinterpret_cast<uint4*>(row0 + mm * ABYTES + ((c ^ rsw) << 4)) = ch[c];
+              }
+              fence_proxy_async_smem();
+              mbar_arrive(&full[s]);
+              if (i + QA < nst)
+#pragma unroll
+                for (int mm = 0; mm < NMAT; ++mm)
+                  ld_q4_pair(rowp[mm] + 36 * (i + QA), raw[j][mm]);
+            }
+          }
+        }
+      }
+    } else {
+      // 16-bit rows: thread m takes chunk c = m % 8 (16 bytes) of rows
+      // 8 (m / 8) + j, j = 0..7, i.e. row j of 8-row group m / 8
+      constexpr int P = umma_ahead16<NMAT>();
+      const int c = m & 7, g = m >> 3;
+      const uint8_t* rowp[NMAT][8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const size_t off = (size_t)max(ids[8 * g + j], 0) * p.rb + (size_t)c * 16;
+        rowp[0][j] = p.wa + off;
+        if constexpr (NMAT == 2) rowp[NMAT - 1][j] = p.wa2 + off;
+      }
+      const uint64_t pol = policy_evict_first();
+      uint4 raw[P][NMAT][8];
+      auto issue = [&](int i, uint4 (&r)[NMAT][8]) {
+#pragma unroll
+        for (int mm = 0; mm < NMAT; ++mm)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) r[mm][j] = ldg_stream_hint(rowp[mm][j] + 128 * i, pol);
+      };
+#pragma unroll
+      for (int j = 0; j < P; ++j)
+        if (j < nst) issue(j, raw[j]);
+      uint8_t* gbase = smem + g * 1024;
+      for (int i0 = 0; i0 < nst && ok; i0 += P) {
+#pragma unroll
+        for (int q = 0; q < P; ++q) {
+          const int i = i0 + q;
+          if (i < nst && ok) {
+            const int s = i % NS;
+            if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
+            if (ok) {
+              uint8_t* st = gbase + (size_t)s * STAGE;
+#pragma unroll
+              for (int mm = 0; mm < NMAT; ++mm)
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  *reinterpret_cast<uint4*>(st + mm * ABYTES + j * 128 + ((c ^ j) << 4)) =
+                      raw[q][mm][j];
+              fence_proxy_async_smem();
+              mbar_arrive(&full[s]);
+              if (i + P < nst) issue(i + P, raw[q]);
+            }
+          }
+        }
+      }
+    }
     // epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (neurons)
     const int quad = warp & 3;
-    const int m = quad * 32 + lane;
-    const bool ok = mbar_wait_sleep(&done, 0);
+    const int mr = quad * 32 + lane;
+    const bool done_ok = mbar_wait_sleep(&done, 0);
     tc_fence_after();
-    const int k = k0 + m;
-    const int id = ids[m];
-    const float bias = bias_s[m];
+    const int k = k0 + mr;
+    const int id = ids[mr];
+    const float bias = bias_s[mr];
 #pragma unroll
     for (int c0 = 0; c0 < N; c0 += 8) {
       uint32_t ra[8], ru[8];
@@ -273,15 +432,16 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           const int n = c0 + j;
           if (n < p.B) {
             float h = 0.f;
-            if (ok && id >= 0) {
+            if (ok && done_ok && id >= 0) {
               const float r = fmaxf(__uint_as_float(ra[j]) + bias, 0.f);
               h = ACT == 1 ? r * __uint_as_float(ru[j]) : ACT == 2 ? r * r : r;
             }
-            const uint16_t hi = to16<DT>(h);
-            const float fh = from16<DT>(hi);
-            if (DT == 0 && isinf(fh)) set_error(kErrRange);
+            constexpr int HT = Q4 ? 0 : DT;  // H is fp16 with fp16 and Q4_0 weights
+            const uint16_t hi = to16<HT>(h);
+            const float fh = from16<HT>(hi);
+            if (HT == 0 && isinf(fh)) set_error(kErrRange);
             p.hh[(size_t)n * p.F + k] = hi;
-            p.hl[(size_t)n * p.F + k] = to16<DT>(h - fh);
+            p.hl[(size_t)n * p.F + k] = to16<HT>(h - fh);
           }
         }
       }
@@ -299,16 +459,23 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 // CTA (c, s) sums the neuron positions of slice s (stages of 64) into the
 // 128 x N accumulator of columns [128c, 128c + 128) and writes it to
 // part[s].  Positions past the list hold H = 0 (the up kernel writes zeros
-// up to the next multiple of 128), and their rows are gathered from row 0.
+// up to the next multiple of 128), and their weight rows are taken from row 0.
+//   warp 0     copies the stage's H tiles, hi and lo (TMA)
+//   warp 1     issues the MMAs and owns the tensor memory
+//   warps 2-5  build the weight operand: 64 neurons x 128 columns per stage,
+//              each neuron's 256-byte row segment read by 16 threads, stored
+//              as one 128-byte row in each of the two column atoms (MN-major,
+//              swizzled); then the epilogue
 template <int DT, int N, int NS>
 __global__ void __launch_bounds__(kUmmaThreads, 1)
-    k_umma_down(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_hh,
-                const __grid_constant__ CUtensorMap tm_hl, UmmaParams p) {
+    k_umma_down(const __grid_constant__ CUtensorMap tm_hh, const __grid_constant__ CUtensorMap tm_hl,
+                UmmaParams p) {
+  constexpr bool Q4 = DT == 2;
   constexpr int ABYTES = kUmmaM * kUmmaK * 2;  // 2 column atoms of 64 neurons x 128 B
   constexpr int BBYTES = N * kUmmaK * 2;
   constexpr int STAGE = umma_down_stage<N>();
   constexpr uint32_t NCOL = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
-  constexpr uint32_t IDESC = idesc_f16<DT, kUmmaM, N, 1, 0>();
+  constexpr uint32_t IDESC = idesc_f16<Q4 ? 0 : DT, kUmmaM, N, 1, 0>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -328,7 +495,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   const int col0 = blockIdx.x * kUmmaM;
   if (t == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + kUmmaM);  // the H copies + 128 builder threads
       mbar_init(&empty[s], 1);
     }
     mbar_init(&done, 1);
@@ -341,41 +508,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   const uint32_t tmem = tmem_base;
 
   if (warp == 0) {
-    // copy engine feeder: the whole warp reads the stage's 64 neuron ids
-    // (two per lane, the next stage's while this one's copies are issued)
-    auto ids_of = [&](int i, int& a, int& b) {
-      const int kp = (st0 + i) * kUmmaK + 2 * lane;
-      a = kp < K ? p.idx[kp] : 0;
-      b = kp + 1 < K ? p.idx[kp + 1] : 0;
-      a = (a < 0 || a >= p.F) ? 0 : a;  // flagged by the up kernel; its H is 0
-      b = (b < 0 || b >= p.F) ? 0 : b;
-    };
-    int na = 0, nb = 0;
-    if (nst > 0) ids_of(0, na, nb);
-    for (int i = 0; i < nst; ++i) {
-      const int s = i % NS;
-      const int ca = na, cb = nb;
-      if (i + 1 < nst) ids_of(i + 1, na, nb);
-      bool ok = true;
-      if (lane == 0) {
-        if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
-        if (ok) mbar_arrive_expect_tx(&full[s], STAGE);
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      uint8_t* st = smem + (size_t)s * STAGE;
-#pragma unroll 1
-      for (int q = 0; q < kUmmaK / 4; ++q) {  // neurons 4q .. 4q+3 of the stage
-        const int r0 = __shfl_sync(0xffffffffu, ca, 2 * q);
-        const int r1 = __shfl_sync(0xffffffffu, cb, 2 * q);
-        const int r2 = __shfl_sync(0xffffffffu, ca, 2 * q + 1);
-        const int r3 = __shfl_sync(0xffffffffu, cb, 2 * q + 1);
-        if (lane == 0) {
-          tma_gather4(st + 512 * q, &tm_w, col0, r0, r1, r2, r3, &full[s]);
-          tma_gather4(st + ABYTES / 2 + 512 * q, &tm_w, col0 + 64, r0, r1, r2, r3, &full[s]);
-        }
-      }
-      if (lane == 0) {
+    if (lane == 0) {  // H tiles
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % NS;
+        if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) break;
+        uint8_t* st = smem + (size_t)s * STAGE;
+        mbar_arrive_expect_tx(&full[s], 2 * BBYTES);
         tma_load2d(st + ABYTES, &tm_hh, (st0 + i) * kUmmaK, 0, &full[s]);
         tma_load2d(st + ABYTES + BBYTES, &tm_hl, (st0 + i) * kUmmaK, 0, &full[s]);
       }
@@ -402,9 +540,117 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     }
     __syncwarp();
   } else {
+    const int m = t - 64;  // 0..127
+    bool ok = true;
+    if constexpr (Q4) {
+      // thread m takes neuron m / 2 of each stage and columns
+      // [64 (m % 2), 64 (m % 2) + 64) of the tile: two blocks, which become one
+      // 128-byte row of column atom m % 2
+      const int kk = m >> 1, half = m & 1;
+      const size_t coff = (size_t)(col0 / 32) * 18 + 36 * half;
+      auto row_of = [&](int i) -> const uint8_t* {
+        const int kp = (st0 + i) * kUmmaK + kk;
+        int id = kp < K ? p.idx[kp] : -1;
+        if (id < 0 || id >= p.F) id = -1;  // flagged by the up kernel; zero row
+        return id < 0 ? nullptr : p.wd + (size_t)id * p.rb + coff;
+      };
+      constexpr int QA = q4_ahead<1>();
+      uint32_t raw[QA][9];
+      bool live[QA];
+#pragma unroll
+      for (int j = 0; j < QA; ++j) {
+        const uint8_t* r = j < nst ? row_of(j) : nullptr;
+        live[j] = r != nullptr;
+        if (r) ld_q4_pair(r, raw[j]);
+      }
+      const uint32_t rsw = (uint32_t)(kk & 7);
+      for (int i0 = 0; i0 < nst && ok; i0 += QA) {
+#pragma unroll
+        for (int j = 0; j < QA; ++j) {
+          const int i = i0 + j;
+          if (i < nst && ok) {
+            const int s = i % NS;
+            if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
+            if (ok) {
+              uint8_t* row0 = smem + (size_t)s * STAGE + half * (ABYTES / 2) + (kk >> 3) * 1024 +
+                              (kk & 7) * 128;
+              uint4 ch[8];
+              if (live[j]) {
+                dq_q4_pair(raw[j], ch);
+              } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) ch[c] = make_uint4(0, 0, 0, 0);
+              }
+#pragma unroll
+              for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(row0 + ((c ^ rsw) << 4)) = ch[c];
+              fence_proxy_async_smem();
+              mbar_arrive(&full[s]);
+              if (i + QA < nst) {
+                const uint8_t* r = row_of(i + QA);
+                live[j] = r != nullptr;
+                if (r) ld_q4_pair(r, raw[j]);
+              }
+            }
+          }
+        }
+      }
+    } else {
+      // 16-bit rows: thread m takes column chunk c = m % 16 (8 columns) of
+      // neurons 8 (m / 16) + j, j = 0..7 of the stage
+      constexpr int P = 2;
+      const int c = m & 15, g = m >> 4;
+      const uint8_t* cbase = p.wd + (size_t)(col0 + 8 * c) * 2;
+      const uint64_t pol = policy_evict_first();
+      auto ids_of = [&](int i, int (&id)[8]) {
+        const int kp = (st0 + i) * kUmmaK + 8 * g;
+        if (kp + 8 <= K) {
+          const int4 a = __ldg(reinterpret_cast<const int4*>(p.idx + kp));
+          const int4 b = __ldg(reinterpret_cast<const int4*>(p.idx + kp + 4));
+          id[0] = a.x; id[1] = a.y; id[2] = a.z; id[3] = a.w;
+          id[4] = b.x; id[5] = b.y; id[6] = b.z; id[7] = b.w;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) id[j] = kp + j < K ? p.idx[kp + j] : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) id[j] = (id[j] < 0 || id[j] >= p.F) ? 0 : id[j];
+      };
+      uint4 raw[P][8];
+      int idn[8];
+      auto issue = [&](int i, uint4 (&r)[8]) {  // ids of stage i are in idn
+#pragma unroll
+        for (int j = 0; j < 8; ++j) r[j] = ldg_stream_hint(cbase + (size_t)idn[j] * p.rb, pol);
+        if (i + 1 < nst) ids_of(i + 1, idn);
+      };
+      if (nst > 0) ids_of(0, idn);
+#pragma unroll
+      for (int j = 0; j < P; ++j)
+        if (j < nst) issue(j, raw[j]);
+      uint8_t* gbase = smem + (c >> 3) * (ABYTES / 2) + g * 1024;
+      const int cc = c & 7;
+      for (int i0 = 0; i0 < nst && ok; i0 += P) {
+#pragma unroll
+        for (int q = 0; q < P; ++q) {
+          const int i = i0 + q;
+          if (i < nst && ok) {
+            const int s = i % NS;
+            if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
+            if (ok) {
+              uint8_t* st = gbase + (size_t)s * STAGE;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(st + j * 128 + ((cc ^ j) << 4)) = raw[q][j];
+              fence_proxy_async_smem();
+              mbar_arrive(&full[s]);
+              if (i + P < nst) issue(i + P, raw[q]);
+            }
+          }
+        }
+      }
+    }
     const int quad = warp & 3;
-    const int c = col0 + quad * 32 + lane;  // output column of this lane
-    const bool ok = nst == 0 || mbar_wait_sleep(&done, 0);
+    const int col = col0 + quad * 32 + lane;  // output column of this lane
+    const bool done_ok = nst == 0 || mbar_wait_sleep(&done, 0);
     tc_fence_after();
 #pragma unroll
     for (int c0 = 0; c0 < N; c0 += 8) {
@@ -416,9 +662,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int n = c0 + j;
-        if (n < p.B && c < p.d)
-          p.part[((size_t)blockIdx.y * p.B + n) * p.d + c] =
-              (nst > 0 && ok) ? __uint_as_float(r[j]) : 0.f;
+        if (n < p.B && col < p.d)
+          p.part[((size_t)blockIdx.y * p.B + n) * p.d + col] =
+              (nst > 0 && ok && done_ok) ? __uint_as_float(r[j]) : 0.f;
       }
     }
   }

@@ -64,6 +64,7 @@ TRAFFIC = {"ratio": 1.070, "src_sha": "24dcaa110b6d3731", "config": "falcon-40b"
 EXTRAS = [
     ("opt-6.7b_b1", "opt-6.7b", 1, 32),
     ("opt-6.7b-sqrelu_b1", "opt-6.7b-sqrelu", 1, 8),
+    ("opt-6.7b-adaptive_b1", "opt-6.7b-adaptive", 1, 32),
     ("relu-llama2-13b_b1", "relu-llama2-13b", 1, 10),
     ("relu-llama2-13b_b8", "relu-llama2-13b", 8, 10),
     ("llama2-70b-q4_b1", "llama2-70b-q4", 1, 10),
@@ -261,8 +262,9 @@ def ffn_launch_bytes(cfg, K, B):
     return K * (nm * rb + 4 + 4) + B * cfg.d_model * 2 + B * cfg.d_model * 4
 
 
-def predictor_bytes(cfg):
-    return cfg.rank * cfg.d_model * 2 + cfg.rank * 4 + cfg.d_ff * cfg.rank * 2 + cfg.d_ff * 4
+def predictor_bytes(cfg, rank=None):
+    r = cfg.rank if rank is None else rank
+    return r * cfg.d_model * 2 + r * 4 + cfg.d_ff * r * 2 + cfg.d_ff * 4
 
 
 # ------------------------------------------------------------------ our arm
@@ -291,10 +293,34 @@ class Stack:
                                     dtype=self.torch.uint8, device="cuda")
         return other
 
+    def hot_first(self):
+        """The same stack with every layer's neurons renumbered hottest first
+        (pi_permute_layer), ordered by the generator's firing profile -- what
+        an offline activation profiler would measure."""
+        import numpy as np
+        torch, pi, synth = self.torch, self.pi, self.synth
+        other = Stack.__new__(Stack)
+        other.__dict__.update(self.__dict__)
+        keys = ("w_up", "w_gate", "w_down_t", "w2", "b2", "b_up", "b_gate")
+        layers = []
+        for l, L in enumerate(self.layers):
+            kw = dict(L.__dict__)
+            for k in keys:
+                v = getattr(L, k)
+                kw[k] = None if v is None else torch.empty_like(v)
+            P = synth.LayerData(**kw)
+            perm = torch.from_numpy(np.argsort(-L.p, kind="stable").astype(np.int32)).cuda()
+            pi.pi_permute_layer(self.arr[l], perm, self.descs([P])[0])
+            layers.append(P)
+        torch.cuda.synchronize()
+        other.layers = layers
+        other.arr = other.descs(layers)
+        return other
+
     def descs(self, ls):
         c = self.cfg
         return self.pi.layer_array([self.pi.layer_from_tensors(
-            d_model=c.d_model, d_ff=c.d_ff, rank=c.rank, wdtype=c.wdtype, adtype=c.adtype,
+            d_model=c.d_model, d_ff=c.d_ff, rank=L.w1.shape[0], wdtype=c.wdtype, adtype=c.adtype,
             act=c.act, w1=L.w1, b1=L.b1, w2=L.w2, b2=L.b2, threshold=L.threshold, w_up=L.w_up,
             w_gate=L.w_gate, w_down_t=L.w_down_t, b_up=L.b_up, b_gate=L.b_gate) for L in ls])
 
@@ -376,8 +402,8 @@ class Stack:
         """Algorithmic bytes of one step: gathered rows and activations (fb_sum)
         plus every layer's predictor and the residual read and written."""
         c = self.cfg
-        return float(fb_sum) + n_batches * c.n_layers * (predictor_bytes(c) +
-                                                        self.B * c.d_model * 4 * 2)
+        per_token = sum(predictor_bytes(c, L.w1.shape[0]) for L in self.layers)
+        return float(fb_sum) + n_batches * (per_token + c.n_layers * self.B * c.d_model * 4 * 2)
 
 
 def measure(stack, T, steps, warmup, peak, barrier=None, seed_offset=0):
@@ -595,6 +621,13 @@ def run_ours(args, rank, world, local):
                 "sample": (f"token 0 of the workload through layers 0-{nl_done - 1} of {NL}, "
                            f"single-threaded C++ fp64 oracle, {per_layer:.3f} s per layer; "
                            f"tokens/s scaled to the {NL}-layer stack")}
+        # ---- hot-row ordering: the same stack renumbered hottest-first
+        if world == 1:
+            hst = st.hot_first()
+            r, _, _ = measure(hst, T, max(3, args.steps // 2), 1, peak)
+            r["speedup_over_profile_order"] = round(r["value"] / value, 4)
+            extras["hot_first"] = r
+            del hst
     del st, X0, Xw
     torch.cuda.empty_cache()
 

@@ -233,6 +233,28 @@ int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_re
                            void* workspace, size_t workspace_bytes, void* stream,
                            void* const* ffn_events);
 
+/*
+ * Hot-row ordering (unite.ai page, "Neuronen-Platzierung und -Verwaltung":
+ * the offline solver places neurons by how often they fire).  One B200 holds
+ * every neuron, so placement becomes an order: this call copies layer `src`
+ * into the caller's buffers of `dst` with its neurons renumbered, neuron i of
+ * dst being neuron perm[i] of src -- hot neurons first when perm sorts them by
+ * firing frequency, so that the rows a token gathers lie closer together.
+ *   - Moved: the rows of W_up, W_gate, W_down^T and W2 and the entries of
+ *     b_up, b_gate and b2.  W1, b1 and the threshold are not touched (dst may
+ *     point at src's).
+ *   - perm   [d_ff] int32 device memory, a permutation of 0..d_ff-1.  An id
+ *            outside [0, d_ff) is flagged in the device error word and its
+ *            destination row left untouched; a repeated id duplicates a
+ *            neuron (not checked).
+ *   - dst    same shapes, dtypes, activation and biases present as src; each
+ *            permuted tensor a device buffer that does not overlap src's.
+ * The permuted layer computes the same function; its index lists name the
+ * new ids (dst id i is src id perm[i]).  Asynchronous on `stream`.
+ */
+int32_t pi_permute_layer(const pi_layer* src, const int32_t* perm, const pi_layer* dst,
+                         void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,6 +29,27 @@ class Config:
     batches: Tuple[int, ...] = (1,)
     n_tokens: int = 128
     prompt_tokens: int = 0
+    # adaptive predictor sizing (unite.ai page, "Adaptive Sparsity-Prädiktoren":
+    # each layer's predictor is sized from that layer's sparsity and skew):
+    # the Zipf exponent runs linearly over [zipf_s - skew_spread, zipf_s +
+    # skew_spread] across the layers, and with adaptive_rank the predictor
+    # rank shrinks where the firing profile is more skewed
+    skew_spread: float = 0.0
+    adaptive_rank: bool = False
+
+    def layer_zipf(self, layer: int) -> float:
+        if self.n_layers <= 1 or self.skew_spread == 0.0:
+            return self.zipf_s
+        return self.zipf_s + self.skew_spread * (2.0 * layer / (self.n_layers - 1) - 1.0)
+
+    def layer_rank(self, layer: int) -> int:
+        """Predictor rank of one layer: the config's rank scaled by
+        (zipf_s / s_layer)^2, a multiple of 16 within [rank / 2, 2 rank]."""
+        if not self.adaptive_rank:
+            return self.rank
+        r = self.rank * (self.zipf_s / self.layer_zipf(layer)) ** 2
+        r = int(round(r / 16.0)) * 16
+        return max(self.rank // 2, min(2 * self.rank, r))
 
     @property
     def seed_weights(self) -> int:
@@ -56,6 +77,10 @@ CONFIGS = {
         # list: ReLU, ReGLU and Squared-ReLU models)
         Config(5, "opt-6.7b-sqrelu", 32, 4096, 16384, "sqrelu", "f16", "f16", 0.02, 1.1, 0.20,
                1024, n_tokens=128),
+        # the OPT-6.7B shapes with a per-layer skew profile (Zipf 0.8 .. 1.4) and
+        # predictors sized per layer (ranks 624 .. 1936)
+        Config(6, "opt-6.7b-adaptive", 32, 4096, 16384, "relu", "f16", "f16", 0.02, 1.1, 0.20,
+               1024, n_tokens=128, skew_spread=0.3, adaptive_rank=True),
     ]
 }
 

@@ -180,7 +180,7 @@ class LayerData:
 def make_layer(cfg: Config, layer: int, device="cpu", mode: str = "R") -> LayerData:
     if mode not in ("R", "F"):
         raise ValueError("mode must be 'R' (recall target) or 'F' (fraction target)")
-    d, F, r = cfg.d_model, cfg.d_ff, cfg.rank
+    d, F, r = cfg.d_model, cfg.d_ff, cfg.layer_rank(layer)
     if r % 2:
         raise ValueError("predictor rank must be even for the +/- construction")
     S = cfg.seed_weights
@@ -233,7 +233,7 @@ def make_layer(cfg: Config, layer: int, device="cpu", mode: str = "R") -> LayerD
     sv = np.maximum(sv, 1e-30)
     rho = cuv / (su * sv)
 
-    p = zipf_profile(F, cfg.zipf_s, cfg.mean_active, _sub_seed(S, layer, _T_PERM))
+    p = zipf_profile(F, cfg.layer_zipf(layer), cfg.mean_active, _sub_seed(S, layer, _T_PERM))
     b = su * ndtri(p)
 
     def frac(delta):

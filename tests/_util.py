@@ -44,7 +44,7 @@ def device_layer(L, device="cuda"):
     Ld = L.to(device)
     c = Ld.cfg
     desc = pi.layer_from_tensors(
-        d_model=c.d_model, d_ff=c.d_ff, rank=c.rank, wdtype=c.wdtype, adtype=c.adtype, act=c.act,
+        d_model=c.d_model, d_ff=c.d_ff, rank=Ld.w1.shape[0], wdtype=c.wdtype, adtype=c.adtype, act=c.act,
         w1=Ld.w1, b1=Ld.b1, w2=Ld.w2, b2=Ld.b2, threshold=Ld.threshold,
         w_up=Ld.w_up, w_gate=Ld.w_gate, w_down_t=Ld.w_down_t, b_up=Ld.b_up, b_gate=Ld.b_gate)
     return Ld, desc

@@ -166,3 +166,28 @@ def test_static_scratch_validates_arguments(lib):
     assert st == pi.binding.PI_ERR_UNSUPPORTED
     st = _status(pi.pi_sparse_ffn_static, _layer(w_down_t=None), FAKE, 1, FAKE, FAKE, FAKE)
     assert st == pi.binding.PI_ERR_INVALID_ARG
+
+
+def test_permute_layer_validation(lib):
+    """pi_permute_layer rejects mismatched layers, a missing perm and a dst
+    tensor that overlaps its src, before touching the device."""
+    E = 1 << 40  # another fake region, far from FAKE
+    src = _layer()
+    dst = _layer(w_up=E, w_down_t=E + (8 << 20), b_up=E + (16 << 20),
+                 pred=_pred(w2=E + (24 << 20), b2=E + (32 << 20)))
+    perm = FAKE
+    assert _status(pi.pi_permute_layer, src, None, dst) == pi.binding.PI_ERR_INVALID_ARG
+    # shapes must match
+    other = _layer(d_model=1024, pred=_pred(d_model=1024), w_up=E, w_down_t=E + (8 << 20),
+                   b_up=E + (16 << 20))
+    assert _status(pi.pi_permute_layer, src, perm, other) == pi.binding.PI_ERR_INVALID_ARG
+    # a bias present on one side only
+    nob = _layer(w_up=E, w_down_t=E + (8 << 20), b_up=None,
+                 pred=_pred(w2=E + (24 << 20), b2=E + (32 << 20)))
+    assert _status(pi.pi_permute_layer, src, perm, nob) == pi.binding.PI_ERR_INVALID_ARG
+    # dst W_up overlapping src W_up (2048 rows of 1 KB from FAKE)
+    ov = _layer(w_up=FAKE + 4096, w_down_t=E + (8 << 20), b_up=E + (16 << 20),
+                pred=_pred(w2=E + (24 << 20), b2=E + (32 << 20)))
+    assert _status(pi.pi_permute_layer, src, perm, ov) == pi.binding.PI_ERR_INVALID_ARG
+    # in place
+    assert _status(pi.pi_permute_layer, src, perm, src) == pi.binding.PI_ERR_INVALID_ARG
