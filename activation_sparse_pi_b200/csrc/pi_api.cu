@@ -87,11 +87,13 @@ size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 #define PI_LDG_CPS 2
 #endif
 int ffn_cps(int B) { return B == 1 ? PI_LDG_CPS : 1; }
+// up to this many partial planes are summed by k_reduce_few
+constexpr int kReduceFew = 16;
 int ffn_grid(int B);
 
 // ------------------------------------------------------------ workspace
 struct WsLayout {
-  size_t bar, a, mask, idx, count, xl, part, h, total;
+  size_t bar, a, mask, umask, idx, count, xl, part, h, total;
 };
 
 int down_slices(int d, int B, int nsm) {
@@ -109,6 +111,7 @@ WsLayout ws_layout(int d, int F, int r, int B) {
   w.bar = o;   o += 256;
   w.a = o;     o += al256((size_t)kAReplicas * B * r * 4);
   w.mask = o;  o += al256((size_t)B * (F / 32) * 4);
+  w.umask = o; o += al256((size_t)(F / 32) * 4);
   w.idx = o;   o += al256((size_t)F * 4);
   w.count = o; o += 256;
   w.xl = o;    o += al256((size_t)B * d * 2);
@@ -228,6 +231,50 @@ int32_t check_ws(void* ws, size_t have, size_t need) {
   if (!aligned16(ws)) return fail(PI_ERR_WORKSPACE, "workspace must be 16-byte aligned");
   if (have < need) return fail(PI_ERR_WORKSPACE, "workspace has %zu bytes, need %zu", have, need);
   return PI_OK;
+}
+
+// ------------------------------------------------- tensor-core batched path
+// Batches of at least kUmmaMinBatch tokens with 16-bit weights run the
+// gathered up and down projections as tcgen05 GEMMs (pi_umma.cuh); their
+// operands are described to the copy engine by tensor maps built here.
+constexpr int kUmmaMinBatch = 8;
+
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// A row-major [rows x inner] tensor of 16-bit values, read in boxes of
+// box_inner x box_rows with the 128-byte swizzle; rows and columns outside the
+// tensor read as zeros.
+bool make_tmap16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool umma_ok(const pi_layer* L, int B) {
+  return B >= kUmmaMinBatch && B <= 64 && L->d_model % kUmmaM == 0 && tmap_encoder() != nullptr;
+}
+
+// pipeline stages that fit two CTAs per SM (at least 2, at most 6)
+constexpr int umma_ns(int stage_bytes) {
+  return (110 * 1024) / stage_bytes < 2 ? 2 : (110 * 1024) / stage_bytes > 6 ? 6
+                                              : (110 * 1024) / stage_bytes;
 }
 
 // ------------------------------------------------------------ predictor
@@ -448,12 +495,59 @@ cudaError_t predict_cpt(const pi_predictor* P, const uint16_t* x, const float* x
   return cudaErrorInvalidValue;
 }
 
+// Predictor layer 2 on the tensor cores (batches of 16 or more, ranks that
+// are a multiple of 64): a as hi + lo 16-bit parts from layer 1, the mask
+// written whole by the kernel's ballots.
+constexpr int kUmmaPredMinBatch = 16;
+
+bool umma_pred_ok(int B, const pi_predictor* P) {
+  return B >= kUmmaPredMinBatch && B <= 64 && P->rank % kUmmaK == 0 && tmap_encoder() != nullptr;
+}
+
+template <int DT, int N>
+cudaError_t launch_umma_pred2_n(const pi_predictor* P, const CUtensorMap& th,
+                                const CUtensorMap& tl, const UmmaPredParams& p, cudaStream_t st) {
+  constexpr int STAGE = kUmmaM * kUmmaK * 2 + 2 * N * kUmmaK * 2;
+  constexpr int NS = umma_ns(STAGE);
+  return launch(k_umma_pred2<DT, N, NS>, dim3((P->d_ff + kUmmaM - 1) / kUmmaM),
+                dim3(kUmmaThreads), (size_t)NS * STAGE + 1024, st, th, tl, p);
+}
+
+template <int DT>
+cudaError_t umma_pred2(const pi_predictor* P, int B, const uint16_t* ah, const uint16_t* al,
+                       uint32_t* mask, uint32_t* umask, float* logits, cudaStream_t st) {
+  const int N = (B + 15) / 16 * 16, r = P->rank;
+  CUtensorMap th{}, tl{};
+  if (!make_tmap16(&th, ah, r, B, (uint64_t)r * 2, kUmmaK, N) ||
+      !make_tmap16(&tl, al, r, B, (uint64_t)r * 2, kUmmaK, N))
+    return cudaErrorInvalidValue;
+  UmmaPredParams p{};
+  p.w2 = static_cast<const uint8_t*>(P->w2);
+  p.b2 = P->b2;
+  p.mask = mask;
+  p.umask = umask;
+  p.logits = logits;
+  p.threshold = P->threshold;
+  p.r = r;
+  p.F = P->d_ff;
+  p.B = B;
+  switch (N) {
+    case 16: return launch_umma_pred2_n<DT, 16>(P, th, tl, p, st);
+    case 32: return launch_umma_pred2_n<DT, 32>(P, th, tl, p, st);
+    case 48: return launch_umma_pred2_n<DT, 48>(P, th, tl, p, st);
+    default: return launch_umma_pred2_n<DT, 64>(P, th, tl, p, st);
+  }
+}
+
 // x16: 16-bit input, or null with xr (residual) given; xo receives x_l then.
 // bar: the workspace's grid-barrier words, zeroed by the API call beforehand.
+// umask (optional): receives the OR of the batch's mask rows when the
+// tensor-core layer 2 runs (returns whether it was written).
 template <int DT>
 int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const float* xr,
                      uint16_t* xo, uint32_t* mask, float* logits, float* a, uint32_t* bar,
-                     cudaStream_t st) {
+                     cudaStream_t st, uint32_t* umask = nullptr, bool* umask_written = nullptr) {
+  if (umask_written) *umask_written = false;
   const int d = P->d_model;
   if (predict_fused_ok(B, P)) {
     const cudaError_t e = B == 1 ? predict_cpt<DT, 1>(P, x16, xr, xo, a, mask, logits, bar, st)
@@ -461,6 +555,11 @@ int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const fl
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "predictor launch failed: %s", cudaGetErrorString(e));
     return PI_OK;
   }
+  // layer 2 on the tensor cores takes a as 16-bit hi + lo parts, written by
+  // layer 1 next to a (the workspace's a region holds several copies of a)
+  const bool tc2 = umma_pred_ok(B, P);
+  uint16_t* ah = reinterpret_cast<uint16_t*>(a + (size_t)B * P->rank);
+  uint16_t* al = ah + (size_t)B * P->rank;
   if (pred1_fused_ok(B, d)) {
     PI_CUDA((pred1_dispatch<DT>(P, B, x16, xr, xo, a, st)));
   } else {
@@ -473,12 +572,19 @@ int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const fl
     p.bias = P->b1;
     p.x16 = x16;
     p.out = a;
+    p.out_hi = tc2 ? ah : nullptr;
+    p.out_lo = tc2 ? al : nullptr;
     p.nrows = P->rank;
     p.len = d;
     p.B = B;
     PI_CUDA((rows_bb<DT, kModePred1>(p, P->rank, st)));
   }
-  if (pred2_fused_ok(B, P->rank)) {
+  if (tc2) {
+    const cudaError_t e = umma_pred2<DT>(P, B, ah, al, mask, umask, logits, st);
+    if (e != cudaSuccess)
+      return fail(PI_ERR_CUDA, "tensor-core predictor launch failed: %s", cudaGetErrorString(e));
+    if (umask_written) *umask_written = umask != nullptr;
+  } else if (pred2_fused_ok(B, P->rank)) {
     if (B == 1) PI_CUDA((pred2_cpl<DT, 1>(P, a, mask, logits, st)));
     else PI_CUDA((pred2_cpl<DT, 2>(P, a, mask, logits, st)));
   } else {
@@ -642,50 +748,6 @@ cudaError_t up_generic_act(const pi_layer* L, int B, const uint16_t* x, const in
   if (L->act == PI_REGLU) return launch_up_generic<WDT, 1>(L, B, x, idx, count, h, st);
   if (L->act == PI_SQRELU) return launch_up_generic<WDT, 2>(L, B, x, idx, count, h, st);
   return launch_up_generic<WDT, 0>(L, B, x, idx, count, h, st);
-}
-
-// ------------------------------------------------- tensor-core batched path
-// Batches of at least kUmmaMinBatch tokens with 16-bit weights run the
-// gathered up and down projections as tcgen05 GEMMs (pi_umma.cuh); their
-// operands are described to the copy engine by tensor maps built here.
-constexpr int kUmmaMinBatch = 8;
-
-PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      f = nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }();
-  return fn;
-}
-
-// A row-major [rows x inner] tensor of 16-bit values, read in boxes of
-// box_inner x box_rows with the 128-byte swizzle; rows and columns outside the
-// tensor read as zeros.
-bool make_tmap16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
-                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
-  auto enc = tmap_encoder();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {inner, rows};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool umma_ok(const pi_layer* L, int B) {
-  return B >= kUmmaMinBatch && B <= 64 && L->d_model % kUmmaM == 0 && tmap_encoder() != nullptr;
-}
-
-// pipeline stages that fit two CTAs per SM (at least 2, at most 6)
-constexpr int umma_ns(int stage_bytes) {
-  return (110 * 1024) / stage_bytes < 2 ? 2 : (110 * 1024) / stage_bytes > 6 ? 6
-                                              : (110 * 1024) / stage_bytes;
 }
 
 template <int DT, int ACT, int N>
@@ -866,6 +928,12 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "batched down launch failed: %s", cudaGetErrorString(e));
   }
   if (ev) PI_CUDA(record_event(ev[1], st));
+  if (G <= kReduceFew) {
+    const dim3 rg((n4 + 255) / 256);
+    if (mode == 0) PI_CUDA((launch(k_reduce_few<0>, rg, dim3(256), 0, st, (const float*)part, G, n4, out)));
+    else PI_CUDA((launch(k_reduce_few<1>, rg, dim3(256), 0, st, (const float*)part, G, n4, out)));
+    return PI_OK;
+  }
   const dim3 rg((n4 + kRedCols - 1) / kRedCols);
   const dim3 rt(kRedCols * kRedSlices);
   if (mode == 0) PI_CUDA((launch(k_reduce<0>, rg, rt, 0, st, (const float*)part, G, n4, out)));
@@ -1027,9 +1095,13 @@ int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_re
     const pi_layer* L = &layers[l];
     int32_t* idx = idx_out ? idx_out + (size_t)l * L->d_ff : reinterpret_cast<int32_t*>(ws + w.idx);
     int32_t* cnt = count_out ? count_out + l : reinterpret_cast<int32_t*>(ws + w.count);
+    uint32_t* umask = reinterpret_cast<uint32_t*>(ws + w.umask);
+    bool have_union = false;
     int32_t s = (L->adtype == PI_F16)
-                    ? predict_impl<0>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, bar, st)
-                    : predict_impl<1>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, bar, st);
+                    ? predict_impl<0>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, bar,
+                                      st, umask, &have_union)
+                    : predict_impl<1>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, bar,
+                                      st, umask, &have_union);
     if (s) return s;
     if (ffn_events && (!ffn_events[2 * l] || !ffn_events[2 * l + 1]))
       return fail(PI_ERR_INVALID_ARG, "ffn_events[%d..%d] must be events", 2 * l, 2 * l + 1);
@@ -1038,6 +1110,9 @@ int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_re
       // compaction fused into the FFN kernel: it reads the mask bits directly
       src = FfnSrc{nullptr, nullptr, mask, (int)batch, idx_out ? idx : nullptr,
                    count_out ? cnt : nullptr, &layers[(l + 1) % n_layers].pred};
+    } else if (have_union) {  // the predictor already ORed the batch's rows
+      PI_CUDA((launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, (const uint32_t*)umask,
+                      1, L->d_ff, idx, cnt)));
     } else {
       PI_CUDA((launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, (const uint32_t*)mask,
                       (int)batch, L->d_ff, idx, cnt)));

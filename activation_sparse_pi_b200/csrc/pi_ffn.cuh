@@ -799,4 +799,27 @@ __global__ void __launch_bounds__(kRedCols * kRedSlices) k_reduce(const float* _
   }
 }
 
+// The same sum for a few partial planes (G small, as from the tensor-core
+// down projection): one thread per float4 column adds the G planes in order.
+template <int MODE>
+__global__ void __launch_bounds__(256) k_reduce_few(const float* __restrict__ part, int G, int n4,
+                                                    float* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  const int col = blockIdx.x * 256 + threadIdx.x;
+  if (col >= n4) return;
+  const float4* src = reinterpret_cast<const float4*>(part);
+  float4 t = src[col];
+  for (int g = 1; g < G; ++g) {
+    const float4 v = src[(size_t)g * n4 + col];
+    t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
+  }
+  float4* o = reinterpret_cast<float4*>(out) + col;
+  if (MODE == 1) {
+    const float4 x = *o;
+    t.x += x.x; t.y += x.y; t.z += x.z; t.w += x.w;
+  }
+  *o = t;
+}
+
 }  // namespace pi

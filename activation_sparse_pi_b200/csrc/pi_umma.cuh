@@ -676,4 +676,169 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   }
 }
 
+// Predictor layer 2 with the threshold, at batches of 16 or more (a dense
+// contraction there): s = W2 a + b2, mask bit = s > threshold.  One CTA per
+// 128 rows of W2 (all rows, no gather), the contraction over the rank in
+// stages of 64.  The hidden activations a (fp32) enter as the hi + lo pair of
+// 16-bit values written by predictor layer 1.  In the epilogue a warp holds
+// 32 consecutive neurons, one per lane, so a ballot over the warp is exactly
+// one mask word per token: the mask is written whole, with no atomics.
+//   warp 0     copies the stage's a tiles, hi and lo (TMA)
+//   warp 1     issues the MMAs and owns the tensor memory
+//   warps 2-5  load the stage's W2 rows (8 threads per 128-byte row piece) into
+//              the swizzled layout; then the epilogue
+struct UmmaPredParams {
+  const uint8_t* w2;       // [F x r] 16-bit rows
+  const float* b2;         // [F]
+  uint32_t* mask;          // [B x F/32]
+  uint32_t* umask;         // [F/32] union of the batch's rows, or null
+  float* logits;           // [B x F] or null
+  float threshold;
+  int r, F, B;
+};
+
+template <int DT, int N, int NS>
+__global__ void __launch_bounds__(kUmmaThreads, 1)
+    k_umma_pred2(const __grid_constant__ CUtensorMap tm_ah, const __grid_constant__ CUtensorMap tm_al,
+                 UmmaPredParams p) {
+  constexpr int ABYTES = kUmmaM * kUmmaK * 2;
+  constexpr int BBYTES = N * kUmmaK * 2;
+  constexpr int STAGE = ABYTES + 2 * BBYTES;
+  constexpr uint32_t NCOL = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+  constexpr uint32_t IDESC = idesc_f16<DT, kUmmaM, N, 0, 0>();
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ uint64_t full[NS], empty[NS], done;
+  __shared__ uint32_t tmem_base;
+
+  pdl_wait();
+  pdl_trigger();
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int row0 = blockIdx.x * kUmmaM;
+  if (t == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1 + kUmmaM);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(&tmem_base, NCOL);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const int nst = p.r / kUmmaK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % NS;
+        if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) break;
+        uint8_t* st = smem + (size_t)s * STAGE;
+        mbar_arrive_expect_tx(&full[s], 2 * BBYTES);
+        tma_load2d(st + ABYTES, &tm_ah, i * kUmmaK, 0, &full[s]);
+        tma_load2d(st + ABYTES + BBYTES, &tm_al, i * kUmmaK, 0, &full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % NS;
+        if (!mbar_wait(&full[s], (i / NS) & 1)) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + (size_t)s * STAGE);
+        const uint32_t sh = sa + ABYTES, sl = sh + BBYTES;
+#pragma unroll
+        for (int kk = 0; kk < kUmmaK / 16; ++kk) {
+          const uint64_t ad = sw128_desc(sa + 32 * kk, 16, 1024);
+          umma_f16(tmem, ad, sw128_desc(sh + 32 * kk, 16, 1024), IDESC, (i | kk) != 0);
+          umma_f16(tmem, ad, sw128_desc(sl + 32 * kk, 16, 1024), IDESC, 1);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(&done);
+    }
+    __syncwarp();
+  } else {
+    const int m = t - 64;
+    const int c = m & 7, g = m >> 3;
+    const size_t rb = (size_t)p.r * 2;
+    const uint8_t* rowp[8];
+    bool live[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int row = row0 + 8 * g + j;
+      live[j] = row < p.F;
+      rowp[j] = p.w2 + (size_t)(live[j] ? row : 0) * rb + (size_t)c * 16;
+    }
+    const uint64_t pol = policy_evict_first();
+    constexpr int P = 2;
+    uint4 raw[P][8];
+    auto issue = [&](int i, uint4 (&rr)[8]) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        rr[j] = live[j] ? ldg_stream_hint(rowp[j] + 128 * i, pol) : make_uint4(0, 0, 0, 0);
+    };
+#pragma unroll
+    for (int j = 0; j < P; ++j)
+      if (j < nst) issue(j, raw[j]);
+    bool ok = true;
+    uint8_t* gbase = smem + g * 1024;
+    for (int i0 = 0; i0 < nst && ok; i0 += P) {
+#pragma unroll
+      for (int q = 0; q < P; ++q) {
+        const int i = i0 + q;
+        if (i < nst && ok) {
+          const int s = i % NS;
+          if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
+          if (ok) {
+            uint8_t* st = gbase + (size_t)s * STAGE;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(st + j * 128 + ((c ^ j) << 4)) = raw[q][j];
+            fence_proxy_async_smem();
+            mbar_arrive(&full[s]);
+            if (i + P < nst) issue(i + P, raw[q]);
+          }
+        }
+      }
+    }
+    // epilogue: lane = neuron 32 (w % 4) + lane of the tile; ballot = mask word
+    const int quad = warp & 3;
+    const int n = row0 + quad * 32 + lane;
+    const bool done_ok = mbar_wait_sleep(&done, 0);
+    tc_fence_after();
+    const float bias = n < p.F ? p.b2[n] : 0.f;
+    uint32_t uni = 0u;  // the union over the batch (the stack's compaction input)
+#pragma unroll
+    for (int c0 = 0; c0 < N; c0 += 8) {
+      uint32_t rr[8];
+      tmem_ld8(tmem + ((uint32_t)(quad * 32) << 16) + c0, rr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int b = c0 + j;
+        if (b < p.B) {  // warp-uniform
+          const float sv = __uint_as_float(rr[j]) + bias;
+          const bool valid = ok && done_ok && n < p.F;
+          if (p.logits && valid) p.logits[(size_t)b * p.F + n] = sv;
+          const uint32_t word = __ballot_sync(0xffffffffu, valid && sv > p.threshold);
+          uni |= word;
+          if (lane == 0 && row0 + quad * 32 < p.F)
+            p.mask[(size_t)b * (p.F / 32) + (row0 + quad * 32) / 32] = word;
+        }
+      }
+    }
+    if (p.umask && lane == 0 && row0 + quad * 32 < p.F) p.umask[(row0 + quad * 32) / 32] = uni;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, NCOL);
+  }
+}
+
 }  // namespace pi

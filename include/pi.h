@@ -117,9 +117,11 @@ const char* pi_status_string(int32_t status);
 const char* pi_last_error(void);
 
 /*
- * Reads and clears the device-side error word (0 = none; nonzero = a kernel
- * gave up on a bounded wait or saw an index outside d_ff).  Synchronises the
- * current device.  Returns PI_OK or PI_ERR_CUDA.
+ * Reads and clears the device-side error word, an OR of: 1 = a kernel gave up
+ * on a bounded wait; 2 = a neuron id outside [0, d_ff) was skipped; 4 = on the
+ * tensor-core batched path with fp16 or Q4_0 weights, an FFN activation
+ * exceeded the fp16 range (|h| > 65504) and the output is not valid.
+ * Synchronises the current device.  Returns PI_OK or PI_ERR_CUDA.
  */
 int32_t pi_device_error(int32_t* code_out);
 
@@ -173,6 +175,11 @@ int32_t pi_compact(const uint32_t* mask_bits, int32_t batch, int32_t d_ff,
  *   y      [batch x d_model] fp32 out (overwritten)
  * The summation order is fixed, so repeated calls give bit-identical y.
  * Passing idx = 0..d_ff-1 and count = d_ff gives the dense FFN.
+ * At batch >= 8 (d_model % 128 == 0) the up and down projections run on the
+ * tensor cores: products of 16-bit operands accumulate in fp32, the
+ * activations h enter the down projection as a hi + lo pair of 16-bit values
+ * (about 16 significant bits with bf16 weights, 22 with fp16), and Q4_0
+ * weights are rounded once to fp16 after dequantization (relative 2^-12).
  */
 int32_t pi_sparse_ffn(const pi_layer* layer, const void* x, int32_t batch,
                       const int32_t* idx, const int32_t* count, float* y,
