@@ -501,53 +501,98 @@ cudaError_t predict_cpt(const pi_predictor* P, const uint16_t* x, const float* x
 constexpr int kUmmaPredMinBatch = 16;
 
 bool umma_pred_ok(int B, const pi_predictor* P) {
-  return B >= kUmmaPredMinBatch && B <= 64 && P->rank % kUmmaK == 0 && tmap_encoder() != nullptr;
+  return B >= kUmmaPredMinBatch && B <= 64 && P->rank % kUmmaK == 0 &&
+         P->d_model % kUmmaK == 0 && tmap_encoder() != nullptr;
 }
 
-template <int DT, int N>
-cudaError_t launch_umma_pred2_n(const pi_predictor* P, const CUtensorMap& th,
-                                const CUtensorMap& tl, const UmmaPredParams& p, cudaStream_t st) {
-  constexpr int STAGE = kUmmaM * kUmmaK * 2 + 2 * N * kUmmaK * 2;
+template <bool L1, int DT, int N>
+cudaError_t launch_umma_pred_n(int rows, int S, const CUtensorMap& t0, const CUtensorMap& t1,
+                               const UmmaPredParams& p, cudaStream_t st) {
+  constexpr int STAGE = kUmmaM * kUmmaK * 2 + (L1 ? 1 : 2) * N * kUmmaK * 2;
   constexpr int NS = umma_ns(STAGE);
-  return launch(k_umma_pred2<DT, N, NS>, dim3((P->d_ff + kUmmaM - 1) / kUmmaM),
-                dim3(kUmmaThreads), (size_t)NS * STAGE + 1024, st, th, tl, p);
+  return launch(k_umma_pred<L1, DT, N, NS>, dim3((rows + kUmmaM - 1) / kUmmaM, S),
+                dim3(kUmmaThreads), (size_t)NS * STAGE + 1024, st, t0, t1, p);
 }
 
+template <bool L1, int DT>
+cudaError_t umma_pred_n(int N, int rows, int S, const CUtensorMap& t0, const CUtensorMap& t1,
+                        const UmmaPredParams& p, cudaStream_t st) {
+  switch (N) {
+    case 16: return launch_umma_pred_n<L1, DT, 16>(rows, S, t0, t1, p, st);
+    case 32: return launch_umma_pred_n<L1, DT, 32>(rows, S, t0, t1, p, st);
+    case 48: return launch_umma_pred_n<L1, DT, 48>(rows, S, t0, t1, p, st);
+    default: return launch_umma_pred_n<L1, DT, 64>(rows, S, t0, t1, p, st);
+  }
+}
+
+// Layer 1 (split over the contraction into `part`, then finished into the
+// hi + lo parts of a) and layer 2 with the threshold.  part_bytes bounds the
+// number of slices.
 template <int DT>
-cudaError_t umma_pred2(const pi_predictor* P, int B, const uint16_t* ah, const uint16_t* al,
-                       uint32_t* mask, uint32_t* umask, float* logits, cudaStream_t st) {
-  const int N = (B + 15) / 16 * 16, r = P->rank;
-  CUtensorMap th{}, tl{};
-  if (!make_tmap16(&th, ah, r, B, (uint64_t)r * 2, kUmmaK, N) ||
+cudaError_t umma_predict(const pi_predictor* P, int B, const uint16_t* x, uint16_t* ah,
+                         uint16_t* al, float* part, size_t part_bytes, uint32_t* mask,
+                         uint32_t* umask, float* logits, cudaStream_t st) {
+  const int N = (B + 15) / 16 * 16, r = P->rank, d = P->d_model;
+  CUtensorMap tx{}, th{}, tl{};
+  if (!make_tmap16(&tx, x, d, B, (uint64_t)d * 2, kUmmaK, N) ||
+      !make_tmap16(&th, ah, r, B, (uint64_t)r * 2, kUmmaK, N) ||
       !make_tmap16(&tl, al, r, B, (uint64_t)r * 2, kUmmaK, N))
     return cudaErrorInvalidValue;
-  UmmaPredParams p{};
-  p.w2 = static_cast<const uint8_t*>(P->w2);
-  p.b2 = P->b2;
-  p.mask = mask;
-  p.umask = umask;
-  p.logits = logits;
-  p.threshold = P->threshold;
-  p.r = r;
-  p.F = P->d_ff;
-  p.B = B;
-  switch (N) {
-    case 16: return launch_umma_pred2_n<DT, 16>(P, th, tl, p, st);
-    case 32: return launch_umma_pred2_n<DT, 32>(P, th, tl, p, st);
-    case 48: return launch_umma_pred2_n<DT, 48>(P, th, tl, p, st);
-    default: return launch_umma_pred2_n<DT, 64>(P, th, tl, p, st);
-  }
+  // layer 1: about two CTAs per SM, at least 8 stages each
+  const int tiles1 = (r + kUmmaM - 1) / kUmmaM;
+  int S = std::max(1, std::min((2 * num_sms()) / tiles1, (d / kUmmaK) / 8));
+  S = (int)std::max<size_t>(1, std::min<size_t>(S, part_bytes / ((size_t)B * r * 4)));
+  UmmaPredParams p1{};
+  p1.w = static_cast<const uint8_t*>(P->w1);
+  p1.part = part;
+  p1.len = d;
+  p1.nrows = r;
+  p1.B = B;
+  cudaError_t e = umma_pred_n<true, DT>(N, r, S, tx, tx, p1, st);
+  if (e != cudaSuccess) return e;
+  e = launch(k_pred1_finish<DT>, dim3((B * r + 255) / 256), dim3(256), 0, st, (const float*)part,
+             S, B, r, P->b1, ah, al);
+  if (e != cudaSuccess) return e;
+  UmmaPredParams p2{};
+  p2.w = static_cast<const uint8_t*>(P->w2);
+  p2.bias = P->b2;
+  p2.mask = mask;
+  p2.umask = umask;
+  p2.logits = logits;
+  p2.threshold = P->threshold;
+  p2.len = r;
+  p2.nrows = P->d_ff;
+  p2.B = B;
+  return umma_pred_n<false, DT>(N, P->d_ff, 1, th, tl, p2, st);
 }
 
 // x16: 16-bit input, or null with xr (residual) given; xo receives x_l then.
 // bar: the workspace's grid-barrier words, zeroed by the API call beforehand.
 // umask (optional): receives the OR of the batch's mask rows when the
 // tensor-core layer 2 runs (returns whether it was written).
+// part / part_bytes: scratch for the tensor-core layer 1's partial sums.
 template <int DT>
 int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const float* xr,
                      uint16_t* xo, uint32_t* mask, float* logits, float* a, uint32_t* bar,
-                     cudaStream_t st, uint32_t* umask = nullptr, bool* umask_written = nullptr) {
+                     cudaStream_t st, float* part, size_t part_bytes,
+                     uint32_t* umask = nullptr, bool* umask_written = nullptr) {
   if (umask_written) *umask_written = false;
+  if (umma_pred_ok(B, P)) {
+    // both layers on the tensor cores; a as 16-bit hi + lo parts in the
+    // workspace's a region (which holds several copies of a)
+    if (xr) {
+      PI_CUDA((launch(k_cast_rms<DT>, dim3(B), dim3(256), 0, st, xr, xo, P->d_model)));
+      x16 = xo;
+    }
+    uint16_t* ah = reinterpret_cast<uint16_t*>(a);
+    uint16_t* al = ah + (size_t)B * P->rank;
+    const cudaError_t e =
+        umma_predict<DT>(P, B, x16, ah, al, part, part_bytes, mask, umask, logits, st);
+    if (e != cudaSuccess)
+      return fail(PI_ERR_CUDA, "tensor-core predictor launch failed: %s", cudaGetErrorString(e));
+    if (umask_written) *umask_written = umask != nullptr;
+    return PI_OK;
+  }
   const int d = P->d_model;
   if (predict_fused_ok(B, P)) {
     const cudaError_t e = B == 1 ? predict_cpt<DT, 1>(P, x16, xr, xo, a, mask, logits, bar, st)
@@ -555,11 +600,6 @@ int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const fl
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "predictor launch failed: %s", cudaGetErrorString(e));
     return PI_OK;
   }
-  // layer 2 on the tensor cores takes a as 16-bit hi + lo parts, written by
-  // layer 1 next to a (the workspace's a region holds several copies of a)
-  const bool tc2 = umma_pred_ok(B, P);
-  uint16_t* ah = reinterpret_cast<uint16_t*>(a + (size_t)B * P->rank);
-  uint16_t* al = ah + (size_t)B * P->rank;
   if (pred1_fused_ok(B, d)) {
     PI_CUDA((pred1_dispatch<DT>(P, B, x16, xr, xo, a, st)));
   } else {
@@ -572,19 +612,12 @@ int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const fl
     p.bias = P->b1;
     p.x16 = x16;
     p.out = a;
-    p.out_hi = tc2 ? ah : nullptr;
-    p.out_lo = tc2 ? al : nullptr;
     p.nrows = P->rank;
     p.len = d;
     p.B = B;
     PI_CUDA((rows_bb<DT, kModePred1>(p, P->rank, st)));
   }
-  if (tc2) {
-    const cudaError_t e = umma_pred2<DT>(P, B, ah, al, mask, umask, logits, st);
-    if (e != cudaSuccess)
-      return fail(PI_ERR_CUDA, "tensor-core predictor launch failed: %s", cudaGetErrorString(e));
-    if (umask_written) *umask_written = umask != nullptr;
-  } else if (pred2_fused_ok(B, P->rank)) {
+  if (pred2_fused_ok(B, P->rank)) {
     if (B == 1) PI_CUDA((pred2_cpl<DT, 1>(P, a, mask, logits, st)));
     else PI_CUDA((pred2_cpl<DT, 2>(P, a, mask, logits, st)));
   } else {
@@ -783,9 +816,8 @@ cudaError_t umma_up_act(const pi_layer* L, int N, const CUtensorMap& tx, const U
 
 // DT: 0 fp16, 1 bf16, 2 Q4_0 weights (pi_umma.cuh).
 template <int DT>
-cudaError_t umma_ffn(const pi_layer* L, int B, const uint16_t* x, const int32_t* idx,
-                     const int32_t* count, uint16_t* hh, uint16_t* hl, float* part, int S,
-                     cudaStream_t st) {
+cudaError_t umma_ffn(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, uint16_t* hh,
+                     uint16_t* hl, float* part, int S, cudaStream_t st) {
   const int d = L->d_model, F = L->d_ff;
   const int N = (B + 15) / 16 * 16;
   const bool reglu = L->act == PI_REGLU;
@@ -795,8 +827,12 @@ cudaError_t umma_ffn(const pi_layer* L, int B, const uint16_t* x, const int32_t*
       !make_tmap16(&tl, hl, F, B, (uint64_t)F * 2, kUmmaK, N))
     return cudaErrorInvalidValue;
   UmmaParams p{};
-  p.idx = idx;
-  p.count = count;
+  p.idx = src.idx;
+  p.count = src.count;
+  p.mask = src.mask;
+  p.mask_rows = src.mask_rows;
+  p.idx_out = src.idx_out;
+  p.count_out = src.count_out;
   p.wa = static_cast<const uint8_t*>(reglu ? L->w_gate : L->w_up);
   p.wa2 = static_cast<const uint8_t*>(L->w_up);
   p.wd = static_cast<const uint8_t*>(L->w_down_t);
@@ -812,6 +848,10 @@ cudaError_t umma_ffn(const pi_layer* L, int B, const uint16_t* x, const int32_t*
                 : L->act == PI_SQRELU ? umma_up_act<DT, 2>(L, N, tx, p, st)
                                       : umma_up_act<DT, 0>(L, N, tx, p, st);
   if (e != cudaSuccess) return e;
+  if (src.mask) {  // the down projection reads the list the up kernel wrote
+    p.idx = src.idx_out;
+    p.count = src.count_out;
+  }
   switch (N) {
     case 16: return launch_umma_down_n<DT, 16>(L, S, th, tl, p, st);
     case 32: return launch_umma_down_n<DT, 32>(L, S, th, tl, p, st);
@@ -871,14 +911,13 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     if (e != cudaSuccess) return fail(PI_ERR_CUDA, "fused FFN launch failed: %s", cudaGetErrorString(e));
     G = ffn_grid(B);
   } else if (umma_ok(L, B)) {
-    if (src.mask) return fail(PI_ERR_UNSUPPORTED, "mask-driven FFN needs the fused kernel");
     uint16_t* hh = reinterpret_cast<uint16_t*>(ws + w.h);
     uint16_t* hl = hh + (size_t)L->d_ff * B;
     G = umma_slices(d, B, num_sms());
     const cudaError_t e =
-        L->wdtype == PI_BF16  ? umma_ffn<1>(L, B, x, src.idx, src.count, hh, hl, part, G, st)
-        : L->wdtype == PI_Q4_0 ? umma_ffn<2>(L, B, x, src.idx, src.count, hh, hl, part, G, st)
-                               : umma_ffn<0>(L, B, x, src.idx, src.count, hh, hl, part, G, st);
+        L->wdtype == PI_BF16  ? umma_ffn<1>(L, B, x, src, hh, hl, part, G, st)
+        : L->wdtype == PI_Q4_0 ? umma_ffn<2>(L, B, x, src, hh, hl, part, G, st)
+                               : umma_ffn<0>(L, B, x, src, hh, hl, part, G, st);
     if (e != cudaSuccess)
       return fail(PI_ERR_CUDA, "tensor-core FFN launch failed: %s", cudaGetErrorString(e));
   } else {
@@ -1015,15 +1054,19 @@ int32_t pi_predict(const pi_predictor* pred, const void* x, int32_t batch, uint3
   if (!aligned16(x) || !aligned16(mask_bits) || (logits && !aligned16(logits)))
     return fail(PI_ERR_INVALID_ARG, "x, mask_bits and logits must be 16-byte aligned");
   const WsLayout w = ws_layout(pred->d_model, pred->d_ff, pred->rank, batch);
-  if (int32_t s = check_ws(workspace, workspace_bytes, w.a + (size_t)kAReplicas * batch * pred->rank * 4)) return s;
-  float* a = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.a);
-  uint32_t* bar = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + w.bar);
+  if (int32_t s = check_ws(workspace, workspace_bytes, w.total)) return s;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* a = reinterpret_cast<float*>(ws + w.a);
+  float* part = reinterpret_cast<float*>(ws + w.part);
+  uint32_t* bar = reinterpret_cast<uint32_t*>(ws + w.bar);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   PI_CUDA(cudaMemsetAsync(bar, 0, 8, st));
   const uint16_t* x16 = static_cast<const uint16_t*>(x);
   if (pred->dtype == PI_F16)
-    return predict_impl<0>(pred, batch, x16, nullptr, nullptr, mask_bits, logits, a, bar, st);
-  return predict_impl<1>(pred, batch, x16, nullptr, nullptr, mask_bits, logits, a, bar, st);
+    return predict_impl<0>(pred, batch, x16, nullptr, nullptr, mask_bits, logits, a, bar, st, part,
+                           w.h - w.part);
+  return predict_impl<1>(pred, batch, x16, nullptr, nullptr, mask_bits, logits, a, bar, st, part,
+                         w.h - w.part);
 }
 
 int32_t pi_compact(const uint32_t* mask_bits, int32_t batch, int32_t d_ff, int32_t* idx,
@@ -1097,11 +1140,12 @@ int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_re
     int32_t* cnt = count_out ? count_out + l : reinterpret_cast<int32_t*>(ws + w.count);
     uint32_t* umask = reinterpret_cast<uint32_t*>(ws + w.umask);
     bool have_union = false;
+    float* part = reinterpret_cast<float*>(ws + w.part);
     int32_t s = (L->adtype == PI_F16)
                     ? predict_impl<0>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, bar,
-                                      st, umask, &have_union)
+                                      st, part, w.h - w.part, umask, &have_union)
                     : predict_impl<1>(&L->pred, batch, nullptr, x_resid, xl, mask, nullptr, a, bar,
-                                      st, umask, &have_union);
+                                      st, part, w.h - w.part, umask, &have_union);
     if (s) return s;
     if (ffn_events && (!ffn_events[2 * l] || !ffn_events[2 * l + 1]))
       return fail(PI_ERR_INVALID_ARG, "ffn_events[%d..%d] must be events", 2 * l, 2 * l + 1);
@@ -1110,9 +1154,11 @@ int32_t pi_ffn_stack_timed(const pi_layer* layers, int32_t n_layers, float* x_re
       // compaction fused into the FFN kernel: it reads the mask bits directly
       src = FfnSrc{nullptr, nullptr, mask, (int)batch, idx_out ? idx : nullptr,
                    count_out ? cnt : nullptr, &layers[(l + 1) % n_layers].pred};
-    } else if (have_union) {  // the predictor already ORed the batch's rows
-      PI_CUDA((launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, (const uint32_t*)umask,
-                      1, L->d_ff, idx, cnt)));
+    } else if (umma_ok(L, batch)) {
+      // compaction fused into the tensor-core up kernel: every CTA scans the
+      // union (ORed by the predictor, or the batch's mask rows) for its tile
+      src = FfnSrc{nullptr, nullptr, have_union ? umask : mask, have_union ? 1 : (int)batch, idx,
+                   cnt, nullptr};
     } else {
       PI_CUDA((launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, (const uint32_t*)mask,
                       (int)batch, L->d_ff, idx, cnt)));

@@ -194,8 +194,12 @@ constexpr int kUmmaM = 128;        // neuron rows (up) / output columns (down) p
 constexpr int kUmmaK = 64;         // contraction elements per stage (one 128-byte row)
 
 struct UmmaParams {
-  const int32_t* idx;      // neuron list (first *count entries)
+  const int32_t* idx;      // neuron list (first *count entries) ...
   const int32_t* count;
+  const uint32_t* mask;    // ... or, up kernel: the predictor's mask rows
+  int mask_rows;           //   [mask_rows x F/32], whose OR is the list; the
+  int32_t* idx_out;        //   tiles' ids are written to idx_out and the
+  int32_t* count_out;      //   length to count_out
   const uint8_t* wa;       // Q4_0 rows (DT 2): activation rows (W_up or W_gate) ...
   const uint8_t* wa2;      // ... W_up rows (ReGLU) ...
   const uint8_t* wd;       // ... and W_down^T rows
@@ -224,6 +228,15 @@ template <int DT>
 __device__ __forceinline__ float from16(uint16_t u) {
   if constexpr (DT == 0) return __half2float(__ushort_as_half(u));
   else return __uint_as_float((uint32_t)u << 16);
+}
+
+// L2 prefetch of the line holding p, kept in the L2 until used: the operand
+// builders ask for the weight pieces of stage i + kPfAhead while they store
+// stage i, so the loads that fill registers (only a stage or two ahead, for
+// want of registers) find their lines in the L2.
+constexpr int kPfAhead = 8;
+__device__ __forceinline__ void prefetch_line(const void* p) {
+  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
 }
 
 // Stages of 16-bit weight chunks the builders keep in flight in registers.
@@ -262,19 +275,68 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   pdl_wait();
   pdl_trigger();
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  int K = *p.count;
-  K = K < 0 ? 0 : (K > p.F ? p.F : K);
   const int k0 = blockIdx.x * kUmmaM;
-  if (k0 >= K) return;  // whole CTA
-  const int rows = min(kUmmaM, K - k0);
-  if (t < kUmmaM) {
-    int id = t < rows ? p.idx[k0 + t] : -1;
-    if (t < rows && (id < 0 || id >= p.F)) {
-      set_error(kErrBadIndex);
-      id = -1;
+  int K;
+  if (p.mask) {
+    // The list is the ascending union of the mask rows; every CTA scans it
+    // (in the stage buffers, not yet in use) and takes ranks [k0, k0 + 128).
+    __shared__ int scan_tmp[33];
+    const int W = p.F / 32;
+    uint32_t* wmask = reinterpret_cast<uint32_t*>(smem);
+    int* wpre = reinterpret_cast<int*>(smem) + W;
+    const int wpt = (W + kUmmaThreads - 1) / kUmmaThreads;
+    int mine = 0;
+    for (int k = 0; k < wpt; ++k) {
+      const int w = t * wpt + k;
+      if (w < W) {
+        uint32_t m = 0u;
+        for (int b = 0; b < p.mask_rows; ++b) m |= p.mask[(size_t)b * W + w];
+        wmask[w] = m;
+        mine += __popc(m);
+      }
     }
-    ids[t] = id;
-    bias_s[t] = (id >= 0 && p.bias) ? p.bias[id] : 0.f;
+    int pos = block_excl_scan<kUmmaThreads>(mine, scan_tmp, K);
+    for (int k = 0; k < wpt; ++k) {
+      const int w = t * wpt + k;
+      if (w < W) {
+        wpre[w] = pos;
+        pos += __popc(wmask[w]);
+      }
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && t == 0) *p.count_out = K;
+    if (k0 >= K) return;  // whole CTA
+    if (t < kUmmaM) {
+      int id = -1;
+      if (k0 + t < K) {
+        const int q = k0 + t;
+        int lo = 0, hi = W - 1;  // the last word whose prefix is <= q
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (wpre[mid] <= q) lo = mid;
+          else hi = mid - 1;
+        }
+        id = lo * 32 + (int)__fns(wmask[lo], 0, q - wpre[lo] + 1);
+        p.idx_out[q] = id;
+      }
+      ids[t] = id;
+      bias_s[t] = (id >= 0 && p.bias) ? p.bias[id] : 0.f;
+    }
+    __syncthreads();  // the scratch is reused as stage buffers below
+  } else {
+    K = *p.count;
+    K = K < 0 ? 0 : (K > p.F ? p.F : K);
+    if (k0 >= K) return;  // whole CTA
+    const int rows = min(kUmmaM, K - k0);
+    if (t < kUmmaM) {
+      int id = t < rows ? p.idx[k0 + t] : -1;
+      if (t < rows && (id < 0 || id >= p.F)) {
+        set_error(kErrBadIndex);
+        id = -1;
+      }
+      ids[t] = id;
+      bias_s[t] = (id >= 0 && p.bias) ? p.bias[id] : 0.f;
+    }
   }
   if (t == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -338,12 +400,18 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 #pragma unroll
           for (int mm = 0; mm < NMAT; ++mm) ld_q4_pair(rowp[mm] + 36 * j, raw[j][mm]);
       const uint32_t rsw = (uint32_t)(m & 7);
+      for (int j = QA; j < kPfAhead && j < nst; ++j)
+#pragma unroll
+        for (int mm = 0; mm < NMAT; ++mm) prefetch_line(rowp[mm] + 36 * j);
       for (int i0 = 0; i0 < nst && ok; i0 += QA) {
 #pragma unroll
         for (int j = 0; j < QA; ++j) {
           const int i = i0 + j;
           if (i < nst && ok) {
             const int s = i % NS;
+            if (i + kPfAhead < nst)
+#pragma unroll
+              for (int mm = 0; mm < NMAT; ++mm) prefetch_line(rowp[mm] + 36 * (i + kPfAhead));
             if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
             if (ok) {
               uint8_t* row0 = smem + (size_t)s * STAGE + (m >> 3) * 1024 + (m & 7) * 128;
@@ -378,6 +446,13 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         if constexpr (NMAT == 2) rowp[NMAT - 1][j] = p.wa2 + off;
       }
       const uint64_t pol = policy_evict_first();
+      // prefetch: thread m asks for row m's 128-byte piece of each stage
+      const uint8_t* pfrow[NMAT];
+      {
+        const size_t off = (size_t)max(ids[m], 0) * p.rb;
+        pfrow[0] = p.wa + off;
+        if constexpr (NMAT == 2) pfrow[NMAT - 1] = p.wa2 + off;
+      }
       uint4 raw[P][NMAT][8];
       auto issue = [&](int i, uint4 (&r)[NMAT][8]) {
 #pragma unroll
@@ -388,6 +463,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 #pragma unroll
       for (int j = 0; j < P; ++j)
         if (j < nst) issue(j, raw[j]);
+      for (int j = P; j < kPfAhead && j < nst; ++j)
+#pragma unroll
+        for (int mm = 0; mm < NMAT; ++mm) prefetch_line(pfrow[mm] + 128 * j);
       uint8_t* gbase = smem + g * 1024;
       for (int i0 = 0; i0 < nst && ok; i0 += P) {
 #pragma unroll
@@ -395,6 +473,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           const int i = i0 + q;
           if (i < nst && ok) {
             const int s = i % NS;
+            if (i + kPfAhead < nst)
+#pragma unroll
+              for (int mm = 0; mm < NMAT; ++mm) prefetch_line(pfrow[mm] + 128 * (i + kPfAhead));
             if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
             if (ok) {
               uint8_t* st = gbase + (size_t)s * STAGE;
@@ -564,12 +645,26 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         if (r) ld_q4_pair(r, raw[j]);
       }
       const uint32_t rsw = (uint32_t)(kk & 7);
+      // prefetch: the first and last byte of this thread's piece of stage
+      // i + kPfAhead (its row id read one stage earlier)
+      auto pf = [&](const uint8_t* r) {
+        if (r) {
+          prefetch_line(r);
+          prefetch_line(r + 35);
+        }
+      };
+      for (int j = QA; j < kPfAhead && j < nst; ++j) pf(row_of(j));
+      const uint8_t* pnext = kPfAhead < nst ? row_of(kPfAhead) : nullptr;
       for (int i0 = 0; i0 < nst && ok; i0 += QA) {
 #pragma unroll
         for (int j = 0; j < QA; ++j) {
           const int i = i0 + j;
           if (i < nst && ok) {
             const int s = i % NS;
+            if (i + kPfAhead < nst) {
+              pf(pnext);
+              pnext = i + kPfAhead + 1 < nst ? row_of(i + kPfAhead + 1) : nullptr;
+            }
             if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
             if (ok) {
               uint8_t* row0 = smem + (size_t)s * STAGE + half * (ABYTES / 2) + (kk >> 3) * 1024 +
@@ -622,6 +717,20 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         for (int j = 0; j < 8; ++j) r[j] = ldg_stream_hint(cbase + (size_t)idn[j] * p.rb, pol);
         if (i + 1 < nst) ids_of(i + 1, idn);
       };
+      // prefetch: thread m asks for the 128-byte half m % 2 of neuron m / 2's
+      // row segment in stage i + kPfAhead (its id read one stage earlier)
+      const int pk = m >> 1;
+      const uint8_t* pcol = p.wd + (size_t)(col0 + 64 * (m & 1)) * 2;
+      auto pf_id = [&](int i) -> int {
+        const int kp = (st0 + i) * kUmmaK + pk;
+        int id = kp < K ? p.idx[kp] : -1;
+        return (id < 0 || id >= p.F) ? -1 : id;
+      };
+      for (int j = P; j < kPfAhead && j < nst; ++j) {
+        const int id = pf_id(j);
+        if (id >= 0) prefetch_line(pcol + (size_t)id * p.rb);
+      }
+      int pnext = kPfAhead < nst ? pf_id(kPfAhead) : -1;
       if (nst > 0) ids_of(0, idn);
 #pragma unroll
       for (int j = 0; j < P; ++j)
@@ -634,6 +743,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           const int i = i0 + q;
           if (i < nst && ok) {
             const int s = i % NS;
+            if (i + kPfAhead < nst) {
+              if (pnext >= 0) prefetch_line(pcol + (size_t)pnext * p.rb);
+              pnext = i + kPfAhead + 1 < nst ? pf_id(i + kPfAhead + 1) : -1;
+            }
             if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
             if (ok) {
               uint8_t* st = gbase + (size_t)s * STAGE;
@@ -676,34 +789,41 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   }
 }
 
-// Predictor layer 2 with the threshold, at batches of 16 or more (a dense
-// contraction there): s = W2 a + b2, mask bit = s > threshold.  One CTA per
-// 128 rows of W2 (all rows, no gather), the contraction over the rank in
-// stages of 64.  The hidden activations a (fp32) enter as the hi + lo pair of
-// 16-bit values written by predictor layer 1.  In the epilogue a warp holds
-// 32 consecutive neurons, one per lane, so a ballot over the warp is exactly
-// one mask word per token: the mask is written whole, with no atomics.
-//   warp 0     copies the stage's a tiles, hi and lo (TMA)
+// The predictor on the tensor cores, at batches of 16 or more (a dense
+// contraction there).  Both layers read every row of their matrix (no
+// gather): one CTA per 128 rows, the contraction in stages of 64.
+//   layer 2 (L1 = false): s = W2 a + b2 and the threshold.  The hidden
+//     activations a (fp32) enter as the hi + lo pair of 16-bit values written
+//     by layer 1.  In the epilogue a warp holds 32 consecutive neurons, one
+//     per lane, so a ballot over the warp is exactly one mask word per token:
+//     the mask is written whole, with no atomics, and so is the OR of the
+//     batch's words (the union the FFN compacts).
+//   layer 1 (L1 = true): W1 x, split over the contraction (gridDim.y slices,
+//     the rank has only rank/128 tiles); each CTA writes its fp32 partial and
+//     k_pred1_finish sums the slices in order and applies b1 and the ReLU.
+//   warp 0     copies the stage's activation tiles (TMA): a hi and lo, or x
 //   warp 1     issues the MMAs and owns the tensor memory
-//   warps 2-5  load the stage's W2 rows (8 threads per 128-byte row piece) into
-//              the swizzled layout; then the epilogue
+//   warps 2-5  load the stage's weight rows (8 threads per 128-byte row piece)
+//              into the swizzled layout; then the epilogue
 struct UmmaPredParams {
-  const uint8_t* w2;       // [F x r] 16-bit rows
-  const float* b2;         // [F]
-  uint32_t* mask;          // [B x F/32]
-  uint32_t* umask;         // [F/32] union of the batch's rows, or null
-  float* logits;           // [B x F] or null
+  const uint8_t* w;        // [nrows x len] 16-bit rows (W2 or W1)
+  const float* bias;       // b2 (layer 2)
+  uint32_t* mask;          // layer 2: [B x nrows/32]
+  uint32_t* umask;         // layer 2: [nrows/32] union of the batch's rows, or null
+  float* logits;           // layer 2: [B x nrows] or null
   float threshold;
-  int r, F, B;
+  float* part;             // layer 1: [gridDim.y x B x nrows] partial W1 x
+  int len, nrows, B;
 };
 
-template <int DT, int N, int NS>
+template <bool L1, int DT, int N, int NS>
 __global__ void __launch_bounds__(kUmmaThreads, 1)
-    k_umma_pred2(const __grid_constant__ CUtensorMap tm_ah, const __grid_constant__ CUtensorMap tm_al,
-                 UmmaPredParams p) {
+    k_umma_pred(const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
+                UmmaPredParams p) {
+  constexpr int NB = L1 ? 1 : 2;  // activation tiles per stage
   constexpr int ABYTES = kUmmaM * kUmmaK * 2;
   constexpr int BBYTES = N * kUmmaK * 2;
-  constexpr int STAGE = ABYTES + 2 * BBYTES;
+  constexpr int STAGE = ABYTES + NB * BBYTES;
   constexpr uint32_t NCOL = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
   constexpr uint32_t IDESC = idesc_f16<DT, kUmmaM, N, 0, 0>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -716,6 +836,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   pdl_trigger();
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int row0 = blockIdx.x * kUmmaM;
+  const int T = p.len / kUmmaK;  // stages of the whole contraction
+  const int st0 = (int)(((long long)T * blockIdx.y) / gridDim.y);
+  const int nst = (int)(((long long)T * (blockIdx.y + 1)) / gridDim.y) - st0;
   if (t == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1 + kUmmaM);
@@ -729,7 +852,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const int nst = p.r / kUmmaK;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -737,9 +859,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         const int s = i % NS;
         if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) break;
         uint8_t* st = smem + (size_t)s * STAGE;
-        mbar_arrive_expect_tx(&full[s], 2 * BBYTES);
-        tma_load2d(st + ABYTES, &tm_ah, i * kUmmaK, 0, &full[s]);
-        tma_load2d(st + ABYTES + BBYTES, &tm_al, i * kUmmaK, 0, &full[s]);
+        mbar_arrive_expect_tx(&full[s], NB * BBYTES);
+        tma_load2d(st + ABYTES, &tm_b0, (st0 + i) * kUmmaK, 0, &full[s]);
+        if constexpr (!L1) tma_load2d(st + ABYTES + BBYTES, &tm_b1, (st0 + i) * kUmmaK, 0, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -754,7 +876,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         for (int kk = 0; kk < kUmmaK / 16; ++kk) {
           const uint64_t ad = sw128_desc(sa + 32 * kk, 16, 1024);
           umma_f16(tmem, ad, sw128_desc(sh + 32 * kk, 16, 1024), IDESC, (i | kk) != 0);
-          umma_f16(tmem, ad, sw128_desc(sl + 32 * kk, 16, 1024), IDESC, 1);
+          if constexpr (!L1) umma_f16(tmem, ad, sw128_desc(sl + 32 * kk, 16, 1024), IDESC, 1);
         }
         umma_commit(&empty[s]);
       }
@@ -764,14 +886,14 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   } else {
     const int m = t - 64;
     const int c = m & 7, g = m >> 3;
-    const size_t rb = (size_t)p.r * 2;
+    const size_t rb = (size_t)p.len * 2;
     const uint8_t* rowp[8];
     bool live[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int row = row0 + 8 * g + j;
-      live[j] = row < p.F;
-      rowp[j] = p.w2 + (size_t)(live[j] ? row : 0) * rb + (size_t)c * 16;
+      live[j] = row < p.nrows;
+      rowp[j] = p.w + (size_t)(live[j] ? row : 0) * rb + (size_t)st0 * 128 + (size_t)c * 16;
     }
     const uint64_t pol = policy_evict_first();
     constexpr int P = 2;
@@ -784,6 +906,11 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 #pragma unroll
     for (int j = 0; j < P; ++j)
       if (j < nst) issue(j, raw[j]);
+    // prefetch: thread m asks for row m's 128-byte piece of stage i + kPfAhead
+    const bool plive = row0 + m < p.nrows;
+    const uint8_t* prow = p.w + (size_t)(plive ? row0 + m : 0) * rb + (size_t)st0 * 128;
+    for (int j = P; j < kPfAhead && j < nst; ++j)
+      if (plive) prefetch_line(prow + 128 * j);
     bool ok = true;
     uint8_t* gbase = smem + g * 1024;
     for (int i0 = 0; i0 < nst && ok; i0 += P) {
@@ -792,6 +919,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         const int i = i0 + q;
         if (i < nst && ok) {
           const int s = i % NS;
+          if (plive && i + kPfAhead < nst) prefetch_line(prow + 128 * (i + kPfAhead));
           if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
           if (ok) {
             uint8_t* st = gbase + (size_t)s * STAGE;
@@ -805,33 +933,52 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         }
       }
     }
-    // epilogue: lane = neuron 32 (w % 4) + lane of the tile; ballot = mask word
+    // epilogue: lane = row 32 (w % 4) + lane of the tile
     const int quad = warp & 3;
     const int n = row0 + quad * 32 + lane;
-    const bool done_ok = mbar_wait_sleep(&done, 0);
+    const bool done_ok = nst == 0 || mbar_wait_sleep(&done, 0);
     tc_fence_after();
-    const float bias = n < p.F ? p.b2[n] : 0.f;
-    uint32_t uni = 0u;  // the union over the batch (the stack's compaction input)
+    if constexpr (L1) {
 #pragma unroll
-    for (int c0 = 0; c0 < N; c0 += 8) {
-      uint32_t rr[8];
-      tmem_ld8(tmem + ((uint32_t)(quad * 32) << 16) + c0, rr);
-      tmem_wait_ld();
+      for (int c0 = 0; c0 < N; c0 += 8) {
+        uint32_t rr[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (nst > 0) {
+          tmem_ld8(tmem + ((uint32_t)(quad * 32) << 16) + c0, rr);
+          tmem_wait_ld();
+        }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int b = c0 + j;
-        if (b < p.B) {  // warp-uniform
-          const float sv = __uint_as_float(rr[j]) + bias;
-          const bool valid = ok && done_ok && n < p.F;
-          if (p.logits && valid) p.logits[(size_t)b * p.F + n] = sv;
-          const uint32_t word = __ballot_sync(0xffffffffu, valid && sv > p.threshold);
-          uni |= word;
-          if (lane == 0 && row0 + quad * 32 < p.F)
-            p.mask[(size_t)b * (p.F / 32) + (row0 + quad * 32) / 32] = word;
+        for (int j = 0; j < 8; ++j) {
+          const int b = c0 + j;
+          if (b < p.B && n < p.nrows)
+            p.part[((size_t)blockIdx.y * p.B + b) * p.nrows + n] =
+                (ok && done_ok) ? __uint_as_float(rr[j]) : 0.f;
         }
       }
+    } else {
+      const float bias = n < p.nrows ? p.bias[n] : 0.f;
+      uint32_t uni = 0u;
+#pragma unroll
+      for (int c0 = 0; c0 < N; c0 += 8) {
+        uint32_t rr[8];
+        tmem_ld8(tmem + ((uint32_t)(quad * 32) << 16) + c0, rr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int b = c0 + j;
+          if (b < p.B) {  // warp-uniform
+            const float sv = __uint_as_float(rr[j]) + bias;
+            const bool valid = ok && done_ok && n < p.nrows;
+            if (p.logits && valid) p.logits[(size_t)b * p.nrows + n] = sv;
+            const uint32_t word = __ballot_sync(0xffffffffu, valid && sv > p.threshold);
+            uni |= word;
+            if (lane == 0 && row0 + quad * 32 < p.nrows)
+              p.mask[(size_t)b * (p.nrows / 32) + (row0 + quad * 32) / 32] = word;
+          }
+        }
+      }
+      if (p.umask && lane == 0 && row0 + quad * 32 < p.nrows)
+        p.umask[(row0 + quad * 32) / 32] = uni;
     }
-    if (p.umask && lane == 0 && row0 + quad * 32 < p.F) p.umask[(row0 + quad * 32) / 32] = uni;
   }
   tc_fence_before();
   __syncthreads();
@@ -839,6 +986,27 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, NCOL);
   }
+}
+
+// Predictor layer 1 from its split-contraction partials: a = relu(sum over
+// the S slices in order + b1), written as the hi + lo 16-bit parts that layer
+// 2 multiplies.  part [S x B x r].
+template <int DT>
+__global__ void __launch_bounds__(256) k_pred1_finish(const float* __restrict__ part, int S, int B,
+                                                      int r, const float* __restrict__ b1,
+                                                      uint16_t* __restrict__ ahi,
+                                                      uint16_t* __restrict__ alo) {
+  pdl_wait();
+  pdl_trigger();
+  const int e = blockIdx.x * 256 + threadIdx.x;
+  if (e >= B * r) return;
+  float z = part[e];
+  for (int y = 1; y < S; ++y) z += part[(size_t)y * B * r + e];
+  if (b1) z += b1[e % r];
+  const float a = fmaxf(z, 0.f);
+  const uint16_t hi = to16<DT>(a);
+  ahi[e] = hi;
+  alo[e] = to16<DT>(a - from16<DT>(hi));
 }
 
 }  // namespace pi
