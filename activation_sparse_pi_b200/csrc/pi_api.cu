@@ -621,18 +621,21 @@ int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const fl
     if (B == 1) PI_CUDA((pred2_cpl<DT, 1>(P, a, mask, logits, st)));
     else PI_CUDA((pred2_cpl<DT, 2>(P, a, mask, logits, st)));
   } else {
-    PI_CUDA(cudaMemsetAsync(mask, 0, (size_t)B * (P->d_ff / 32) * 4, st));
-    RowsParams p{};
-    p.w = static_cast<const uint8_t*>(P->w2);
-    p.bias = P->b2;
-    p.x32 = a;
-    p.out = logits;
+    // one CTA per mask word and 8 tokens; the rank in 4 (rank <= 1024) or 8
+    // warp groups, so a lane's slice of a stays in registers
+    Pred2WordsParams p{};
+    p.w2 = static_cast<const uint8_t*>(P->w2);
+    p.b2 = P->b2;
+    p.a = a;
     p.mask = mask;
+    p.logits = logits;
     p.threshold = P->threshold;
-    p.nrows = P->d_ff;
-    p.len = P->rank;
+    p.F = P->d_ff;
+    p.r = P->rank;
     p.B = B;
-    PI_CUDA((rows_bb<DT, kModePred2>(p, P->d_ff, st)));
+    const dim3 grid(P->d_ff / 32, (B + 7) / 8);
+    if (P->rank <= 1024) PI_CUDA((launch(k_pred2_words<DT, 4>, grid, dim3(256), 0, st, p)));
+    else PI_CUDA((launch(k_pred2_words<DT, 8>, grid, dim3(256), 0, st, p)));
   }
   return PI_OK;
 }
@@ -799,7 +802,7 @@ cudaError_t launch_umma_down_n(const pi_layer* L, int S, const CUtensorMap& th,
                                const CUtensorMap& tl, const UmmaParams& p, cudaStream_t st) {
   constexpr int STAGE = umma_down_stage<N>();
   constexpr int NS = umma_ns(STAGE);
-  return launch(k_umma_down<DT, N, NS>, dim3(L->d_model / kUmmaM, S), dim3(kUmmaThreads),
+  return launch(k_umma_down<DT, N, NS>, dim3(L->d_model / kUmmaM, S), dim3(kUmmaDownThreads),
                 (size_t)NS * STAGE + 1024, st, th, tl, p);
 }
 

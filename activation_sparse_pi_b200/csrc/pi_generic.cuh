@@ -203,6 +203,97 @@ __global__ void __launch_bounds__(256) k_rows(RowsParams p) {
   }
 }
 
+// ------------------------------------ predictor layer 2, batches of 3 to 15
+// One CTA per mask word: rows 32w .. 32w + 31 of W2 (one contiguous slab,
+// asked of the L2 before the dependency wait) for 8 tokens of the batch
+// (blockIdx.y selects the 8).  The rank is split over NQ warp groups so that
+// each lane holds its slice of a for the 8 tokens in registers (64 floats)
+// and streams one 16-byte chunk of each row; the NQ partial dots of a row
+// meet in shared memory and are added in a fixed order.  Each warp of the
+// combine step holds one token and the 32 rows of the word, so one ballot is
+// the token's mask word: the mask is written whole, with no atomics.
+struct Pred2WordsParams {
+  const uint8_t* w2;       // [F x r] 16-bit rows
+  const float* b2;         // [F]
+  const float* a;          // [B x r] fp32
+  uint32_t* mask;          // [B x F/32]
+  float* logits;           // [B x F] or null
+  float threshold;
+  int F, r, B;
+};
+
+template <int DT, int NQ>
+__global__ void __launch_bounds__(256) k_pred2_words(Pred2WordsParams p) {
+  constexpr int RS = 8 / NQ;          // row streams
+  constexpr int ROWS = 32 / RS;       // rows per warp
+  constexpr int U = 4;                // rows whose chunks are in flight together
+  __shared__ float part[32][NQ][8];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int q = warp % NQ, rs = warp / NQ;
+  const int word = blockIdx.x, b0 = blockIdx.y * 8;
+  const size_t rb = (size_t)p.r * 2;
+  const uint8_t* slab = p.w2 + (size_t)word * 32 * rb;
+  if (t == 0) {  // the word's 32 rows, contiguous: stream them into the L2 now
+    const size_t bytes = 32 * rb;
+    for (size_t o = 0; o < bytes; o += 32768)
+      prefetch_l2(slab + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768));
+  }
+  pdl_wait();
+  pdl_trigger();
+  const int nch = p.r / 8;
+  const int c0 = (int)(((long long)nch * q) / NQ), c1 = (int)(((long long)nch * (q + 1)) / NQ);
+  const int c = c0 + lane;
+  const bool mine = c < c1;  // at most 32 chunks per group (rank <= 2048)
+  float av[8][8];
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    const bool ok = mine && b0 + b < p.B;
+    const float4* ap = reinterpret_cast<const float4*>(p.a + (size_t)(b0 + b) * p.r + (size_t)c * 8);
+    const float4 lo = ok ? __ldg(ap) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 hi = ok ? __ldg(ap + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+    av[b][0] = lo.x; av[b][1] = lo.y; av[b][2] = lo.z; av[b][3] = lo.w;
+    av[b][4] = hi.x; av[b][5] = hi.y; av[b][6] = hi.z; av[b][7] = hi.w;
+  }
+  for (int r0 = 0; r0 < ROWS; r0 += U) {
+    uint4 w[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int row = rs * ROWS + r0 + u;
+      w[u] = mine ? ldg_stream(slab + (size_t)row * rb + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float v[8];
+      const uint32_t wv[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        float z = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack2<DT>(wv[e]);
+          z = fmaf(f.x, av[b][2 * e], z);
+          z = fmaf(f.y, av[b][2 * e + 1], z);
+        }
+        v[b] = z;
+      }
+      const float tot = warp_reduce_transposed<8>(v);  // lane holds token lane / 4
+      if ((lane & 3) == 0) part[rs * ROWS + r0 + u][q][lane >> 2] = tot;
+    }
+  }
+  __syncthreads();
+  // warp b: token b0 + b, lane = row of the word
+  const int b = warp, n = word * 32 + lane;
+  if (b0 + b < p.B) {  // warp-uniform
+    float sv = 0.f;
+#pragma unroll
+    for (int g = 0; g < NQ; ++g) sv += part[lane][g][b];
+    sv += p.b2[n];
+    if (p.logits) p.logits[(size_t)(b0 + b) * p.F + n] = sv;
+    const uint32_t bits = __ballot_sync(0xffffffffu, sv > p.threshold);
+    if (lane == 0) p.mask[(size_t)(b0 + b) * (p.F / 32) + word] = bits;
+  }
+}
+
 // ---------------------------------------------------- batched gathered down
 // Grid (column slices, neuron slices).  Thread: 8 consecutive columns.  For
 // each group of 8 tokens, sums h[k][b] * W_down^T[idx[k]][cols] over the

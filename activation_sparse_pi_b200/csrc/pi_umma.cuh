@@ -190,6 +190,7 @@ __host__ __device__ constexpr int q4_ahead() { return NMAT == 1 ? 4 : 2; }
 
 // ---------------------------------------------------------------- kernels
 constexpr int kUmmaThreads = 192;  // warp 0 copies, warp 1 MMAs, warps 2-5 epilogue
+constexpr int kUmmaDownThreads = 224;  // the down kernel adds warp 6, its L2 prefetcher
 constexpr int kUmmaM = 128;        // neuron rows (up) / output columns (down) per tile
 constexpr int kUmmaK = 64;         // contraction elements per stage (one 128-byte row)
 
@@ -256,7 +257,7 @@ __host__ __device__ constexpr int umma_ahead16() { return NMAT == 1 ? 2 : 1; }
 //              a warp instruction reads four whole 128-byte row pieces) stored
 //              in the swizzled layout; then the epilogue
 template <int DT, int ACT, int N, int NS>
-__global__ void __launch_bounds__(kUmmaThreads, 1)
+__global__ void __launch_bounds__(kUmmaThreads, 2)
     k_umma_up(const __grid_constant__ CUtensorMap tm_x, UmmaParams p) {
   constexpr int NMAT = ACT == 1 ? 2 : 1;
   constexpr bool Q4 = DT == 2;
@@ -387,51 +388,67 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const int m = t - 64;  // 0..127
     bool ok = true;
     if constexpr (Q4) {
-      // thread m builds row m: two Q4_0 blocks (36 bytes) per stage
+      // thread m builds row m.  It loads a super-stage at a time: eight
+      // blocks = 144 bytes = four MMA stages of its row, with nine 128-bit
+      // loads (row pieces of 144 bytes stay 16-byte aligned since d % 256 ==
+      // 0), and decodes two blocks per stage from registers.  (Loading two
+      // blocks per stage as nine 32-bit words made every warp instruction
+      // touch 32 rows for 4 bytes each, and the L1 request rate, not HBM,
+      // set the pace.)  The L2 is asked for the pieces two super-stages ahead.
       const int id = max(ids[m], 0);
       const uint8_t* rowp[NMAT];
       rowp[0] = p.wa + (size_t)id * p.rb;
       if constexpr (NMAT == 2) rowp[NMAT - 1] = p.wa2 + (size_t)id * p.rb;
-      constexpr int QA = q4_ahead<NMAT>();
-      uint32_t raw[QA][NMAT][9];
+      const int nss = nst / 4;  // super-stages
+      constexpr int SSA = kPfAhead / 4;
+      auto pf_ss = [&](int ss) {
 #pragma unroll
-      for (int j = 0; j < QA; ++j)
-        if (j < nst)
-#pragma unroll
-          for (int mm = 0; mm < NMAT; ++mm) ld_q4_pair(rowp[mm] + 36 * j, raw[j][mm]);
+        for (int mm = 0; mm < NMAT; ++mm) {
+          prefetch_line(rowp[mm] + 144 * ss);
+          prefetch_line(rowp[mm] + 144 * ss + 143);
+        }
+      };
+      for (int ss = 1; ss <= SSA && ss < nss; ++ss) pf_ss(ss);
       const uint32_t rsw = (uint32_t)(m & 7);
-      for (int j = QA; j < kPfAhead && j < nst; ++j)
+      uint32_t raw[NMAT][36];
+      auto ld_ss = [&](int ss) {
 #pragma unroll
-        for (int mm = 0; mm < NMAT; ++mm) prefetch_line(rowp[mm] + 36 * j);
-      for (int i0 = 0; i0 < nst && ok; i0 += QA) {
+        for (int mm = 0; mm < NMAT; ++mm) {
+          const uint4* src = reinterpret_cast<const uint4*>(rowp[mm] + 144 * ss);
 #pragma unroll
-        for (int j = 0; j < QA; ++j) {
-          const int i = i0 + j;
-          if (i < nst && ok) {
-            const int s = i % NS;
-            if (i + kPfAhead < nst)
-#pragma unroll
-              for (int mm = 0; mm < NMAT; ++mm) prefetch_line(rowp[mm] + 36 * (i + kPfAhead));
-            if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
-            if (ok) {
-              uint8_t* row0 = smem + (size_t)s * STAGE + (m >> 3) * 1024 + (m & 7) * 128;
-#pragma unroll
-              for (int mm = 0; mm < NMAT; ++mm) {
-                uint4 ch[8];
-                dq_q4_pair(raw[j][mm], ch);
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                  *reinterpret_cast<uint4*>(row0 + mm * ABYTES + ((c ^ rsw) << 4)) = ch[c];
-              }
-              fence_proxy_async_smem();
-              mbar_arrive(&full[s]);
-              if (i + QA < nst)
-#pragma unroll
-                for (int mm = 0; mm < NMAT; ++mm)
-                  ld_q4_pair(rowp[mm] + 36 * (i + QA), raw[j][mm]);
-            }
+          for (int k = 0; k < 9; ++k) {
+            const uint4 v = __ldg(src + k);
+            raw[mm][4 * k] = v.x; raw[mm][4 * k + 1] = v.y;
+            raw[mm][4 * k + 2] = v.z; raw[mm][4 * k + 3] = v.w;
           }
         }
+      };
+      if (nss > 0) ld_ss(0);
+      for (int ss = 0; ss < nss && ok; ++ss) {
+        if (ss + SSA + 1 < nss) pf_ss(ss + SSA + 1);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = 4 * ss + u;
+          const int s = i % NS;
+          if (ok && i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
+          if (ok) {
+            uint8_t* row0 = smem + (size_t)s * STAGE + (m >> 3) * 1024 + (m & 7) * 128;
+#pragma unroll
+            for (int mm = 0; mm < NMAT; ++mm) {
+              uint32_t w[9];
+#pragma unroll
+              for (int k = 0; k < 9; ++k) w[k] = raw[mm][9 * u + k];
+              uint4 ch[8];
+              dq_q4_pair(w, ch);
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(row0 + mm * ABYTES + ((c ^ rsw) << 4)) = ch[c];
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&full[s]);
+          }
+        }
+        if (ss + 1 < nss && ok) ld_ss(ss + 1);
       }
     } else {
       // 16-bit rows: thread m takes chunk c = m % 8 (16 bytes) of rows
@@ -547,8 +564,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 //              each neuron's 256-byte row segment read by 16 threads, stored
 //              as one 128-byte row in each of the two column atoms (MN-major,
 //              swizzled); then the epilogue
+//   warp 6     reads the neuron ids of the stages ahead and asks the L2 for
+//              their row segments, at most kPfAhead stages ahead of the MMAs
+//              (which publish their progress in shared memory); the ids it
+//              reads are then in the L1 for the builders
 template <int DT, int N, int NS>
-__global__ void __launch_bounds__(kUmmaThreads, 1)
+__global__ void __launch_bounds__(kUmmaDownThreads, 2)
     k_umma_down(const __grid_constant__ CUtensorMap tm_hh, const __grid_constant__ CUtensorMap tm_hl,
                 UmmaParams p) {
   constexpr bool Q4 = DT == 2;
@@ -562,10 +583,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
                                              ~uintptr_t(1023));
   __shared__ uint64_t full[NS], empty[NS], done;
   __shared__ uint32_t tmem_base;
+  __shared__ int prog;  // the last stage whose operands the MMA thread has seen
 
   pdl_wait();
   pdl_trigger();
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  if (t == 0) prog = -1;
   int K = *p.count;
   K = K < 0 ? 0 : (K > p.F ? p.F : K);
   const int T = (K + kUmmaK - 1) / kUmmaK;  // stages of the whole list
@@ -604,6 +627,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       for (int i = 0; i < nst; ++i) {
         const int s = i % NS;
         if (!mbar_wait(&full[s], (i / NS) & 1)) break;
+        *reinterpret_cast<volatile int*>(&prog) = i;
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + (size_t)s * STAGE);
         const uint32_t sh = sa + ABYTES, sl = sh + BBYTES;
@@ -620,6 +644,35 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       umma_commit(&done);
     }
     __syncwarp();
+  } else if (warp == 6) {
+    // the L2 prefetcher: lane l takes neurons 2l and 2l + 1 of each stage
+    const size_t coff = Q4 ? (size_t)(col0 / 32) * 18 : (size_t)col0 * 2;
+    const int span = Q4 ? 71 : 255;  // last byte of a neuron's segment
+    for (int j = 0; j < nst; ++j) {
+      uint32_t it = 0;
+      while (*reinterpret_cast<volatile int*>(&prog) < j - kPfAhead && ++it < kWaitLimitSleep)
+        __nanosleep(128);
+      if (it >= kWaitLimitSleep) break;  // only a hint: stop prefetching
+      const int kp = (st0 + j) * kUmmaK + 2 * lane;
+      int ia = -1, ib = -1;
+      if (kp + 1 < K) {
+        const int2 v = __ldg(reinterpret_cast<const int2*>(p.idx + kp));
+        ia = v.x;
+        ib = v.y;
+      } else if (kp < K) {
+        ia = p.idx[kp];
+      }
+      if (ia >= 0 && ia < p.F) {
+        const uint8_t* r = p.wd + (size_t)ia * p.rb + coff;
+        prefetch_line(r);
+        prefetch_line(r + span);
+      }
+      if (ib >= 0 && ib < p.F) {
+        const uint8_t* r = p.wd + (size_t)ib * p.rb + coff;
+        prefetch_line(r);
+        prefetch_line(r + span);
+      }
+    }
   } else {
     const int m = t - 64;  // 0..127
     bool ok = true;
@@ -645,26 +698,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         if (r) ld_q4_pair(r, raw[j]);
       }
       const uint32_t rsw = (uint32_t)(kk & 7);
-      // prefetch: the first and last byte of this thread's piece of stage
-      // i + kPfAhead (its row id read one stage earlier)
-      auto pf = [&](const uint8_t* r) {
-        if (r) {
-          prefetch_line(r);
-          prefetch_line(r + 35);
-        }
-      };
-      for (int j = QA; j < kPfAhead && j < nst; ++j) pf(row_of(j));
-      const uint8_t* pnext = kPfAhead < nst ? row_of(kPfAhead) : nullptr;
       for (int i0 = 0; i0 < nst && ok; i0 += QA) {
 #pragma unroll
         for (int j = 0; j < QA; ++j) {
           const int i = i0 + j;
           if (i < nst && ok) {
             const int s = i % NS;
-            if (i + kPfAhead < nst) {
-              pf(pnext);
-              pnext = i + kPfAhead + 1 < nst ? row_of(i + kPfAhead + 1) : nullptr;
-            }
             if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
             if (ok) {
               uint8_t* row0 = smem + (size_t)s * STAGE + half * (ABYTES / 2) + (kk >> 3) * 1024 +
@@ -717,20 +756,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         for (int j = 0; j < 8; ++j) r[j] = ldg_stream_hint(cbase + (size_t)idn[j] * p.rb, pol);
         if (i + 1 < nst) ids_of(i + 1, idn);
       };
-      // prefetch: thread m asks for the 128-byte half m % 2 of neuron m / 2's
-      // row segment in stage i + kPfAhead (its id read one stage earlier)
-      const int pk = m >> 1;
-      const uint8_t* pcol = p.wd + (size_t)(col0 + 64 * (m & 1)) * 2;
-      auto pf_id = [&](int i) -> int {
-        const int kp = (st0 + i) * kUmmaK + pk;
-        int id = kp < K ? p.idx[kp] : -1;
-        return (id < 0 || id >= p.F) ? -1 : id;
-      };
-      for (int j = P; j < kPfAhead && j < nst; ++j) {
-        const int id = pf_id(j);
-        if (id >= 0) prefetch_line(pcol + (size_t)id * p.rb);
-      }
-      int pnext = kPfAhead < nst ? pf_id(kPfAhead) : -1;
       if (nst > 0) ids_of(0, idn);
 #pragma unroll
       for (int j = 0; j < P; ++j)
@@ -743,10 +768,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           const int i = i0 + q;
           if (i < nst && ok) {
             const int s = i % NS;
-            if (i + kPfAhead < nst) {
-              if (pnext >= 0) prefetch_line(pcol + (size_t)pnext * p.rb);
-              pnext = i + kPfAhead + 1 < nst ? pf_id(i + kPfAhead + 1) : -1;
-            }
             if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
             if (ok) {
               uint8_t* st = gbase + (size_t)s * STAGE;
@@ -817,7 +838,7 @@ struct UmmaPredParams {
 };
 
 template <bool L1, int DT, int N, int NS>
-__global__ void __launch_bounds__(kUmmaThreads, 1)
+__global__ void __launch_bounds__(kUmmaThreads, 2)
     k_umma_pred(const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
                 UmmaPredParams p) {
   constexpr int NB = L1 ? 1 : 2;  // activation tiles per stage
