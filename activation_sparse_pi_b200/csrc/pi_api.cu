@@ -272,9 +272,13 @@ bool umma_ok(const pi_layer* L, int B) {
 }
 
 // pipeline stages that fit two CTAs per SM (at least 2, at most 6)
+#ifndef PI_UMMA_SMEM_KB
+#define PI_UMMA_SMEM_KB 110
+#endif
 constexpr int umma_ns(int stage_bytes) {
-  return (110 * 1024) / stage_bytes < 2 ? 2 : (110 * 1024) / stage_bytes > 6 ? 6
-                                              : (110 * 1024) / stage_bytes;
+  return (PI_UMMA_SMEM_KB * 1024) / stage_bytes < 2 ? 2
+         : (PI_UMMA_SMEM_KB * 1024) / stage_bytes > 6 ? 6
+                                                      : (PI_UMMA_SMEM_KB * 1024) / stage_bytes;
 }
 
 // ------------------------------------------------------------ predictor
@@ -786,6 +790,9 @@ cudaError_t up_generic_act(const pi_layer* L, int B, const uint16_t* x, const in
   return launch_up_generic<WDT, 0>(L, B, x, idx, count, h, st);
 }
 
+// The up projection (grid: p.ucap units or the tiles of all F neurons,
+// whichever is more) and, when its contraction may be split, the kernel
+// that completes split tiles.
 template <int DT, int ACT, int N>
 cudaError_t launch_umma_up_n(const pi_layer* L, const CUtensorMap& tx, const UmmaParams& p,
                              cudaStream_t st) {
@@ -793,8 +800,10 @@ cudaError_t launch_umma_up_n(const pi_layer* L, const CUtensorMap& tx, const Umm
   constexpr int STAGE = umma_up_stage<NMAT, N>();
   constexpr int NS = umma_ns(STAGE);
   const int tiles = (L->d_ff + kUmmaM - 1) / kUmmaM;
-  return launch(k_umma_up<DT, ACT, N, NS>, dim3(tiles), dim3(kUmmaThreads),
-                (size_t)NS * STAGE + 1024, st, tx, p);
+  cudaError_t e = launch(k_umma_up<DT, ACT, N, NS>, dim3(std::max(tiles, p.ucap)),
+                         dim3(kUmmaThreads), (size_t)NS * STAGE + 1024, st, tx, p);
+  if (e != cudaSuccess || p.ucap < 2) return e;
+  return launch(k_umma_up_finish<DT, ACT>, dim3(2 * num_sms()), dim3(256), 0, st, p);
 }
 
 template <int DT, int N>
@@ -820,7 +829,7 @@ cudaError_t umma_up_act(const pi_layer* L, int N, const CUtensorMap& tx, const U
 // DT: 0 fp16, 1 bf16, 2 Q4_0 weights (pi_umma.cuh).
 template <int DT>
 cudaError_t umma_ffn(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src, uint16_t* hh,
-                     uint16_t* hl, float* part, int S, cudaStream_t st) {
+                     uint16_t* hl, float* part, size_t part_bytes, int S, cudaStream_t st) {
   const int d = L->d_model, F = L->d_ff;
   const int N = (B + 15) / 16 * 16;
   const bool reglu = L->act == PI_REGLU;
@@ -844,6 +853,13 @@ cudaError_t umma_ffn(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& 
   p.hh = hh;
   p.hl = hl;
   p.part = part;
+  // a split up projection keeps its slices' sums in the partial-sum scratch,
+  // which the down projection overwrites only after they have been added
+  const int nsm = num_sms();
+  const size_t unit_bytes = (size_t)(reglu ? 2 : 1) * B * kUmmaM * 4;
+  p.pu = part;
+  p.slots = 2 * nsm;
+  p.ucap = (int)std::min<size_t>((size_t)(4 * nsm), part_bytes / unit_bytes);
   p.d = d;
   p.F = F;
   p.B = B;
@@ -917,10 +933,11 @@ int32_t ffn_impl(const pi_layer* L, int B, const uint16_t* x, const FfnSrc& src,
     uint16_t* hh = reinterpret_cast<uint16_t*>(ws + w.h);
     uint16_t* hl = hh + (size_t)L->d_ff * B;
     G = umma_slices(d, B, num_sms());
+    const size_t pb = w.h - w.part;
     const cudaError_t e =
-        L->wdtype == PI_BF16  ? umma_ffn<1>(L, B, x, src, hh, hl, part, G, st)
-        : L->wdtype == PI_Q4_0 ? umma_ffn<2>(L, B, x, src, hh, hl, part, G, st)
-                               : umma_ffn<0>(L, B, x, src, hh, hl, part, G, st);
+        L->wdtype == PI_BF16  ? umma_ffn<1>(L, B, x, src, hh, hl, part, pb, G, st)
+        : L->wdtype == PI_Q4_0 ? umma_ffn<2>(L, B, x, src, hh, hl, part, pb, G, st)
+                               : umma_ffn<0>(L, B, x, src, hh, hl, part, pb, G, st);
     if (e != cudaSuccess)
       return fail(PI_ERR_CUDA, "tensor-core FFN launch failed: %s", cudaGetErrorString(e));
   } else {

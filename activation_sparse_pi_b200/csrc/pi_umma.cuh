@@ -137,14 +137,20 @@ __device__ __forceinline__ void ld_q4_pair(const uint8_t* p, uint32_t (&w)[9]) {
 
 // Two fp16 values (q - 8) * scale for the nibbles q held in two bytes of v
 // (each byte 0..15; sel picks them: 0x4140 bytes 0-1, 0x4342 bytes 2-3).
-// Bits and half2 values are converted with intrinsics, not pointer casts.
-__device__ __forceinline__ uint32_t q4_h2(uint32_t v, uint32_t sel, __half2 scale2) {
-  const uint32_t biased = __byte_perm(v, 0x64646464u, sel);  // halves 0x6400 | q = 1024 + q
-  const __half2 qb = __halves2half2(__ushort_as_half((unsigned short)(biased & 0xffffu)),
-                                    __ushort_as_half((unsigned short)(biased >> 16)));
-  const __half2 r = __hmul2(__hsub2(qb, __float2half2_rn(1032.f)), scale2);
-  return (uint32_t)__half_as_ushort(__low2half(r)) |
-         ((uint32_t)__half_as_ushort(__high2half(r)) << 16);
+// The pair stays packed in one 32-bit register: a byte permute makes the
+// halves 0x6400 | q = 1024 + q, a packed subtract of 1032 leaves q - 8
+// exactly, and a packed multiply by the scale pair rounds once.  (Unpacking
+// to two halves and repacking cost about three times the instructions, and
+// the operand builders were issue-bound on it.)
+__device__ __forceinline__ uint32_t q4_h2(uint32_t v, uint32_t sel, uint32_t scale2) {
+  const uint32_t biased = __byte_perm(v, 0x64646464u, sel);
+  uint32_t r;
+  asm("{\n\t.reg .b32 t;\n\t"
+      "sub.rn.f16x2 t, %1, %3;\n\t"
+      "mul.rn.f16x2 %0, t, %2;\n\t}"
+      : "=r"(r)
+      : "r"(biased), "r"(scale2), "r"(0x64086408u));
+  return r;
 }
 
 // 36 bytes = blocks A and B -> chunks c = 0..7 of 8 consecutive values each
@@ -164,8 +170,7 @@ __device__ __forceinline__ void dq_q4_pair(const uint32_t (&w)[9], uint4 (&out)[
 #pragma unroll
       for (int k = 0; k < 4; ++k) nb[k] = w[5 + k];
     }
-    const __half s = __ushort_as_half((unsigned short)sbits);
-    const __half2 s2 = __halves2half2(s, s);
+    const uint32_t s2 = sbits | (sbits << 16);  // the block scale in both halves
     uint32_t lo[4], hi[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -209,8 +214,32 @@ struct UmmaParams {
   uint16_t* hh;            // [B x F] 16-bit hi part of H (token-major)
   uint16_t* hl;            // [B x F] 16-bit lo part
   float* part;             // down: [gridDim.y x B x d] partial y
+  float* pu;               // up, contraction split in S slices: per (tile, slice)
+                           //   unit, [NMAT x B x 128] fp32 accumulators
+  int ucap;                // up: most units (grid size, room in pu)
+  int slots;               // up: CTAs resident at once (two per SM)
   int d, F, B;
 };
+
+// Slices of the contraction per 128-row tile of the up projection.  With T
+// tiles listed, S slices give T * S units of 1/S of a tile's work each; the
+// pick minimises ceil(T S / slots) / S (waves times the work of a unit) over
+// S = 1..8 (ties to fewer slices), with T S <= ucap and at least 8 stages in
+// a slice.  Slices are whole granules of gran stages.  The up kernel and its
+// finishing kernel both call this, so they agree on S.
+__host__ __device__ inline int up_slices(int T, int ucap, int slots, int ngran, int gran) {
+  int best = 1;
+  long long bw = (T + slots - 1) / slots;  // waves with one slice
+  for (int S = 2; S <= 8; ++S) {
+    if ((long long)T * S > ucap || (ngran / S) * gran < 8) break;
+    const long long w = ((long long)T * S + slots - 1) / slots;
+    if (w * best < bw * S) {
+      best = S;
+      bw = w;
+    }
+  }
+  return best;
+}
 
 // Bytes of one pipeline stage.
 template <int NMAT, int N>
@@ -235,18 +264,53 @@ __device__ __forceinline__ float from16(uint16_t u) {
 // builders ask for the weight pieces of stage i + kPfAhead while they store
 // stage i, so the loads that fill registers (only a stage or two ahead, for
 // want of registers) find their lines in the L2.
-constexpr int kPfAhead = 8;
+#ifndef PI_PF_AHEAD
+#define PI_PF_AHEAD 8
+#endif
+#ifndef PI_PF_EVICT_LAST
+#define PI_PF_EVICT_LAST 1
+#endif
+constexpr int kPfAhead = PI_PF_AHEAD;
 __device__ __forceinline__ void prefetch_line(const void* p) {
+#if PI_PF_EVICT_LAST
   asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
+#else
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+#endif
 }
 
 // Stages of 16-bit weight chunks the builders keep in flight in registers.
+#ifndef PI_UP_AHEAD
+#define PI_UP_AHEAD 2
+#endif
 template <int NMAT>
-__host__ __device__ constexpr int umma_ahead16() { return NMAT == 1 ? 2 : 1; }
+__host__ __device__ constexpr int umma_ahead16() { return NMAT == 1 ? PI_UP_AHEAD : 1; }
 
-// Gathered up projection + activation.  One CTA per tile of 128 listed
-// neurons (tiles past the device-side count exit at once); the contraction
-// runs over d in stages of 64.  DT: 0 fp16, 1 bf16 (weights and tokens),
+// One activation of the up projection: h = act(a + bias) (ReGLU: times the
+// up row's sum u), written as the hi and lo 16-bit parts of H (type HT) at
+// token n, list position k; zero where the position holds no neuron.
+template <int HT, int ACT>
+__device__ __forceinline__ void up_store(const UmmaParams& p, int n, int k, float a, float u,
+                                         float bias, bool live) {
+  float h = 0.f;
+  if (live) {
+    const float r = fmaxf(a + bias, 0.f);
+    h = ACT == 1 ? r * u : ACT == 2 ? r * r : r;
+  }
+  const uint16_t hi = to16<HT>(h);
+  const float fh = from16<HT>(hi);
+  if (HT == 0 && isinf(fh)) set_error(kErrRange);
+  p.hh[(size_t)n * p.F + k] = hi;
+  p.hl[(size_t)n * p.F + k] = to16<HT>(h - fh);
+}
+
+// Gathered up projection + activation.  The work is T tiles of 128 listed
+// neurons (T from the device-side count), each split into S slices of the
+// contraction over d (up_slices: S > 1 when T alone would leave SMs idle);
+// CTA u takes tile u / S, slice u % S, and CTAs past T S exit at once.  A
+// slice runs in stages of 64 elements.  With S = 1 the CTA applies the
+// activation itself; with S > 1 it writes its raw sums to pu and
+// k_umma_up_finish completes the tile.  DT: 0 fp16, 1 bf16 (weights and tokens),
 // 2 Q4_0 weights with fp16 tokens.  ACT: 0 ReLU, 1 ReGLU (gate rows in p.wa,
 // up rows in p.wa2), 2 Squared-ReLU.  N: tokens per MMA (the batch rounded up
 // to a multiple of 16).
@@ -276,15 +340,16 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
   pdl_wait();
   pdl_trigger();
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int k0 = blockIdx.x * kUmmaM;
   int K;
+  // mask mode: the list is the ascending union of the mask rows; every CTA
+  // scans it (in the stage buffers, not yet in use)
+  const uint32_t* wmask = reinterpret_cast<const uint32_t*>(smem);
+  const int* wpre = reinterpret_cast<const int*>(smem) + p.F / 32;
   if (p.mask) {
-    // The list is the ascending union of the mask rows; every CTA scans it
-    // (in the stage buffers, not yet in use) and takes ranks [k0, k0 + 128).
     __shared__ int scan_tmp[33];
     const int W = p.F / 32;
-    uint32_t* wmask = reinterpret_cast<uint32_t*>(smem);
-    int* wpre = reinterpret_cast<int*>(smem) + W;
+    uint32_t* wm = reinterpret_cast<uint32_t*>(smem);
+    int* wp = reinterpret_cast<int*>(smem) + W;
     const int wpt = (W + kUmmaThreads - 1) / kUmmaThreads;
     int mine = 0;
     for (int k = 0; k < wpt; ++k) {
@@ -292,7 +357,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       if (w < W) {
         uint32_t m = 0u;
         for (int b = 0; b < p.mask_rows; ++b) m |= p.mask[(size_t)b * W + w];
-        wmask[w] = m;
+        wm[w] = m;
         mine += __popc(m);
       }
     }
@@ -300,45 +365,51 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
     for (int k = 0; k < wpt; ++k) {
       const int w = t * wpt + k;
       if (w < W) {
-        wpre[w] = pos;
-        pos += __popc(wmask[w]);
+        wp[w] = pos;
+        pos += __popc(wm[w]);
       }
     }
     __syncthreads();
     if (blockIdx.x == 0 && t == 0) *p.count_out = K;
-    if (k0 >= K) return;  // whole CTA
-    if (t < kUmmaM) {
-      int id = -1;
-      if (k0 + t < K) {
-        const int q = k0 + t;
-        int lo = 0, hi = W - 1;  // the last word whose prefix is <= q
+  } else {
+    K = *p.count;
+    K = K < 0 ? 0 : (K > p.F ? p.F : K);
+  }
+  // this CTA's unit: tile of 128 listed neurons, slice of the contraction
+  constexpr int GRAN = Q4 ? 4 : 1;  // Q4_0 rows are read 4 stages (144 B) at a time
+  const int ngran = p.d / kUmmaK / GRAN;
+  const int T = (K + kUmmaM - 1) / kUmmaM;
+  const int S = up_slices(T, p.ucap, p.slots, ngran, GRAN);
+  const int tile = blockIdx.x / S, slice = blockIdx.x - tile * S;
+  if (tile >= T) return;  // whole CTA
+  const int k0 = tile * kUmmaM;
+  const int st0 = ngran * slice / S * GRAN;
+  const int nst = ngran * (slice + 1) / S * GRAN - st0;
+  if (t < kUmmaM) {
+    int id = -1;
+    if (k0 + t < K) {
+      const int q = k0 + t;
+      if (p.mask) {
+        int lo = 0, hi = p.F / 32 - 1;  // the last word whose prefix is <= q
         while (lo < hi) {
           const int mid = (lo + hi + 1) >> 1;
           if (wpre[mid] <= q) lo = mid;
           else hi = mid - 1;
         }
         id = lo * 32 + (int)__fns(wmask[lo], 0, q - wpre[lo] + 1);
-        p.idx_out[q] = id;
+        if (slice == 0) p.idx_out[q] = id;
+      } else {
+        id = p.idx[q];
+        if (id < 0 || id >= p.F) {
+          set_error(kErrBadIndex);
+          id = -1;
+        }
       }
-      ids[t] = id;
-      bias_s[t] = (id >= 0 && p.bias) ? p.bias[id] : 0.f;
     }
-    __syncthreads();  // the scratch is reused as stage buffers below
-  } else {
-    K = *p.count;
-    K = K < 0 ? 0 : (K > p.F ? p.F : K);
-    if (k0 >= K) return;  // whole CTA
-    const int rows = min(kUmmaM, K - k0);
-    if (t < kUmmaM) {
-      int id = t < rows ? p.idx[k0 + t] : -1;
-      if (t < rows && (id < 0 || id >= p.F)) {
-        set_error(kErrBadIndex);
-        id = -1;
-      }
-      ids[t] = id;
-      bias_s[t] = (id >= 0 && p.bias) ? p.bias[id] : 0.f;
-    }
+    ids[t] = id;
+    bias_s[t] = (id >= 0 && p.bias) ? p.bias[id] : 0.f;
   }
+  __syncthreads();  // the scan scratch is reused as stage buffers below
   if (t == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1 + kUmmaM);  // the token copy + 128 builder threads
@@ -352,7 +423,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const int nst = p.d / kUmmaK;
 
   if (warp == 0) {
     if (lane == 0) {  // token tiles
@@ -360,7 +430,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
         const int s = i % NS;
         if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) break;
         mbar_arrive_expect_tx(&full[s], N * kUmmaK * 2);
-        tma_load2d(smem + (size_t)s * STAGE + NMAT * ABYTES, &tm_x, i * kUmmaK, 0, &full[s]);
+        tma_load2d(smem + (size_t)s * STAGE + NMAT * ABYTES, &tm_x, (st0 + i) * kUmmaK, 0,
+                   &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -396,9 +467,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       // touch 32 rows for 4 bytes each, and the L1 request rate, not HBM,
       // set the pace.)  The L2 is asked for the pieces two super-stages ahead.
       const int id = max(ids[m], 0);
+      const size_t roff = (size_t)id * p.rb + (size_t)(st0 / 4) * 144;  // the slice's first block
       const uint8_t* rowp[NMAT];
-      rowp[0] = p.wa + (size_t)id * p.rb;
-      if constexpr (NMAT == 2) rowp[NMAT - 1] = p.wa2 + (size_t)id * p.rb;
+      rowp[0] = p.wa + roff;
+      if constexpr (NMAT == 2) rowp[NMAT - 1] = p.wa2 + roff;
       const int nss = nst / 4;  // super-stages
       constexpr int SSA = kPfAhead / 4;
       auto pf_ss = [&](int ss) {
@@ -458,7 +530,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       const uint8_t* rowp[NMAT][8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const size_t off = (size_t)max(ids[8 * g + j], 0) * p.rb + (size_t)c * 16;
+        const size_t off = (size_t)max(ids[8 * g + j], 0) * p.rb + (size_t)st0 * 128 + (size_t)c * 16;
         rowp[0][j] = p.wa + off;
         if constexpr (NMAT == 2) rowp[NMAT - 1][j] = p.wa2 + off;
       }
@@ -466,7 +538,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       // prefetch: thread m asks for row m's 128-byte piece of each stage
       const uint8_t* pfrow[NMAT];
       {
-        const size_t off = (size_t)max(ids[m], 0) * p.rb;
+        const size_t off = (size_t)max(ids[m], 0) * p.rb + (size_t)st0 * 128;
         pfrow[0] = p.wa + off;
         if constexpr (NMAT == 2) pfrow[NMAT - 1] = p.wa2 + off;
       }
@@ -518,29 +590,34 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
     const int k = k0 + mr;
     const int id = ids[mr];
     const float bias = bias_s[mr];
+    // with S > 1 slices the unit's raw sums go to pu[unit] ([NMAT x B x 128]);
+    // k_umma_up_finish adds the slices and applies the activation
+    float* pu = p.pu + (size_t)blockIdx.x * NMAT * p.B * kUmmaM;
 #pragma unroll
     for (int c0 = 0; c0 < N; c0 += 8) {
       uint32_t ra[8], ru[8];
       tmem_ld8(tmem + ((uint32_t)(quad * 32) << 16) + c0, ra);
       if constexpr (NMAT == 2) tmem_ld8(tmem + ((uint32_t)(quad * 32) << 16) + N + c0, ru);
       tmem_wait_ld();
-      if (k < p.F) {
+      if (S > 1) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int n = c0 + j;
           if (n < p.B) {
-            float h = 0.f;
-            if (ok && done_ok && id >= 0) {
-              const float r = fmaxf(__uint_as_float(ra[j]) + bias, 0.f);
-              h = ACT == 1 ? r * __uint_as_float(ru[j]) : ACT == 2 ? r * r : r;
-            }
-            constexpr int HT = Q4 ? 0 : DT;  // H is fp16 with fp16 and Q4_0 weights
-            const uint16_t hi = to16<HT>(h);
-            const float fh = from16<HT>(hi);
-            if (HT == 0 && isinf(fh)) set_error(kErrRange);
-            p.hh[(size_t)n * p.F + k] = hi;
-            p.hl[(size_t)n * p.F + k] = to16<HT>(h - fh);
+            const bool live = ok && done_ok;
+            pu[(size_t)n * kUmmaM + mr] = live ? __uint_as_float(ra[j]) : 0.f;
+            if constexpr (NMAT == 2)
+              pu[(size_t)(p.B + n) * kUmmaM + mr] = live ? __uint_as_float(ru[j]) : 0.f;
           }
+        }
+      } else if (k < p.F) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int n = c0 + j;
+          if (n < p.B)
+            up_store<Q4 ? 0 : DT, ACT>(p, n, k, __uint_as_float(ra[j]),
+                                       NMAT == 2 ? __uint_as_float(ru[j]) : 0.f, bias,
+                                       ok && done_ok && id >= 0);
         }
       }
     }
@@ -550,6 +627,45 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, NCOL);
+  }
+}
+
+// Completes a split up projection: for every listed position k of the T
+// tiles and token n, adds the S slices' sums in slice order, applies bias
+// and activation and writes H (up_store).  Recomputes S as the up kernel
+// did, and exits at once when S = 1.  Grid-stride over T x B x 128.
+template <int DT, int ACT>
+__global__ void __launch_bounds__(256) k_umma_up_finish(UmmaParams p) {
+  constexpr int NMAT = ACT == 1 ? 2 : 1;
+  constexpr int GRAN = DT == 2 ? 4 : 1;
+  pdl_wait();
+  pdl_trigger();
+  int K = *(p.mask ? p.count_out : p.count);
+  K = K < 0 ? 0 : (K > p.F ? p.F : K);
+  const int T = (K + kUmmaM - 1) / kUmmaM;
+  const int S = up_slices(T, p.ucap, p.slots, p.d / kUmmaK / GRAN, GRAN);
+  if (S == 1) return;
+  const int32_t* list = p.mask ? p.idx_out : p.idx;
+  const size_t total = (size_t)T * p.B * kUmmaM;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (size_t)gridDim.x * blockDim.x) {
+    const int m = (int)(e % kUmmaM);
+    const int n = (int)((e / kUmmaM) % p.B);
+    const int tile = (int)(e / ((size_t)kUmmaM * p.B));
+    const int k = tile * kUmmaM + m;
+    if (k >= p.F) continue;
+    int id = k < K ? list[k] : -1;
+    if (id < 0 || id >= p.F) id = -1;  // a bad id was flagged by the up kernel
+    float a = 0.f, u = 0.f;
+    if (id >= 0) {
+      for (int sl = 0; sl < S; ++sl) {
+        const float* src = p.pu + (size_t)(tile * S + sl) * NMAT * p.B * kUmmaM;
+        a += src[(size_t)n * kUmmaM + m];
+        if constexpr (NMAT == 2) u += src[(size_t)(p.B + n) * kUmmaM + m];
+      }
+    }
+    const float bias = (id >= 0 && p.bias) ? p.bias[id] : 0.f;
+    up_store<DT == 2 ? 0 : DT, ACT>(p, n, k, a, u, bias, id >= 0);
   }
 }
 

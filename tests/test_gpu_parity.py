@@ -33,6 +33,9 @@ SMALL = {
         Config(16, "t-sqrelu-f16", 3, 1024, 4096, "sqrelu", "f16", "f16", 0.02, 1.1, 0.15, 256),
         Config(17, "t-sqrelu-bf16-2560", 2, 2560, 2048, "sqrelu", "bf16", "bf16", 0.02, 1.1, 0.15, 256),
         Config(18, "t-q4-sqrelu", 2, 512, 2048, "sqrelu", "q4_0", "f16", 0.015, 1.1, 0.1, 128),
+        # d = 2048: 32 stages, enough for the batched up projection to split
+        # its contraction (slices of whole 144-byte Q4_0 row pieces)
+        Config(20, "t-q4-reglu-2048", 2, 2048, 2048, "reglu", "q4_0", "f16", 0.015, 1.1, 0.1, 128),
         # per-layer skew and predictor rank (ranks 480, 304, 208, 160)
         Config(19, "t-adaptive-rank", 4, 1024, 4096, "relu", "f16", "f16", 0.02, 1.1, 0.15, 256,
                skew_spread=0.3, adaptive_rank=True),
