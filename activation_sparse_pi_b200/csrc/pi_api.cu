@@ -271,14 +271,15 @@ bool umma_ok(const pi_layer* L, int B) {
   return B >= kUmmaMinBatch && B <= 64 && L->d_model % kUmmaM == 0 && tmap_encoder() != nullptr;
 }
 
-// pipeline stages that fit two CTAs per SM (at least 2, at most 6)
-#ifndef PI_UMMA_SMEM_KB
-#define PI_UMMA_SMEM_KB 110
-#endif
-constexpr int umma_ns(int stage_bytes) {
-  return (PI_UMMA_SMEM_KB * 1024) / stage_bytes < 2 ? 2
-         : (PI_UMMA_SMEM_KB * 1024) / stage_bytes > 6 ? 6
-                                                      : (PI_UMMA_SMEM_KB * 1024) / stage_bytes;
+// Pipeline stages (at least 2, at most 6) within a shared-memory budget
+// that keeps two CTAs on an SM.  16-bit operands arrive by asynchronous
+// copies, which land in the stage buffers: the whole budget goes to stages.
+// Q4_0 operands are loaded through the L1 and decoded in registers, and
+// fewer stages leave the L1 more room for loads in flight (measured: 75 KB
+// beats 110 KB by 12-15% there, and loses by as much on 16-bit rows).
+constexpr int umma_ns(int stage_bytes, bool q4 = false) {
+  const int budget = (q4 ? 75 : 110) * 1024;
+  return budget / stage_bytes < 2 ? 2 : budget / stage_bytes > 6 ? 6 : budget / stage_bytes;
 }
 
 // ------------------------------------------------------------ predictor
@@ -798,7 +799,7 @@ cudaError_t launch_umma_up_n(const pi_layer* L, const CUtensorMap& tx, const Umm
                              cudaStream_t st) {
   constexpr int NMAT = ACT == 1 ? 2 : 1;
   constexpr int STAGE = umma_up_stage<NMAT, N>();
-  constexpr int NS = umma_ns(STAGE);
+  constexpr int NS = umma_ns(STAGE, DT == 2);
   const int tiles = (L->d_ff + kUmmaM - 1) / kUmmaM;
   cudaError_t e = launch(k_umma_up<DT, ACT, N, NS>, dim3(std::max(tiles, p.ucap)),
                          dim3(kUmmaThreads), (size_t)NS * STAGE + 1024, st, tx, p);
@@ -810,7 +811,7 @@ template <int DT, int N>
 cudaError_t launch_umma_down_n(const pi_layer* L, int S, const CUtensorMap& th,
                                const CUtensorMap& tl, const UmmaParams& p, cudaStream_t st) {
   constexpr int STAGE = umma_down_stage<N>();
-  constexpr int NS = umma_ns(STAGE);
+  constexpr int NS = umma_ns(STAGE, DT == 2);
   return launch(k_umma_down<DT, N, NS>, dim3(L->d_model / kUmmaM, S), dim3(kUmmaDownThreads),
                 (size_t)NS * STAGE + 1024, st, th, tl, p);
 }

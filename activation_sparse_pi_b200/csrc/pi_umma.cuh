@@ -188,14 +188,12 @@ __device__ __forceinline__ void dq_q4_pair(const uint32_t (&w)[9], uint4 (&out)[
   }
 }
 
-// Stages of raw Q4_0 blocks the operand builders keep in flight in registers
-// (per thread: NMAT x 36 bytes per stage).
-template <int NMAT>
-__host__ __device__ constexpr int q4_ahead() { return NMAT == 1 ? 4 : 2; }
-
 // ---------------------------------------------------------------- kernels
 constexpr int kUmmaThreads = 192;  // warp 0 copies, warp 1 MMAs, warps 2-5 epilogue
 constexpr int kUmmaDownThreads = 224;  // the down kernel adds warp 6, its L2 prefetcher
+// Stages of raw Q4_0 blocks the down kernel's builders keep in flight in
+// registers (36 bytes per thread per stage).
+constexpr int kQ4DownAhead = 4;
 constexpr int kUmmaM = 128;        // neuron rows (up) / output columns (down) per tile
 constexpr int kUmmaK = 64;         // contraction elements per stage (one 128-byte row)
 
@@ -261,30 +259,38 @@ __device__ __forceinline__ float from16(uint16_t u) {
 }
 
 // L2 prefetch of the line holding p, kept in the L2 until used: the operand
-// builders ask for the weight pieces of stage i + kPfAhead while they store
-// stage i, so the loads that fill registers (only a stage or two ahead, for
-// want of registers) find their lines in the L2.
-#ifndef PI_PF_AHEAD
-#define PI_PF_AHEAD 8
-#endif
-#ifndef PI_PF_EVICT_LAST
-#define PI_PF_EVICT_LAST 1
-#endif
-constexpr int kPfAhead = PI_PF_AHEAD;
+// builders ask for the weight pieces of stage i + kPfAhead while they work on
+// stage i, so the copies and loads of a stage find their lines in the L2.
+// (Measured on the batched kernels: dropping it costs about 30%; longer
+// distances, bursts of a row's pieces and plain eviction priority gain
+// nothing.)
+constexpr int kPfAhead = 8;
 __device__ __forceinline__ void prefetch_line(const void* p) {
-#if PI_PF_EVICT_LAST
   asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
-#else
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-#endif
 }
 
-// Stages of 16-bit weight chunks the builders keep in flight in registers.
-#ifndef PI_UP_AHEAD
-#define PI_UP_AHEAD 2
-#endif
-template <int NMAT>
-__host__ __device__ constexpr int umma_ahead16() { return NMAT == 1 ? PI_UP_AHEAD : 1; }
+// 16-byte asynchronous copy global -> shared that bypasses the L1 (so the
+// bytes in flight are bounded by the pipeline's stage buffers, not by the L1
+// left over after the shared-memory carve-out), and the arrive on an
+// mbarrier once all of this thread's earlier copies have landed (.noinc: the
+// barrier's expected count includes these arrivals).  The consumer fences
+// the async proxy after its wait, before the tensor cores read the stage.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Same, reading src_bytes (0 or 16) and filling the rest of the 16 with zeros.
+__device__ __forceinline__ void cp_async16_fill(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 
 // One activation of the up projection: h = act(a + bias) (ReGLU: times the
 // up row's sum u), written as the hi and lo 16-bit parts of H (type HT) at
@@ -317,9 +323,9 @@ __device__ __forceinline__ void up_store(const UmmaParams& p, int n, int k, floa
 //   warp 0     copies the stage's token tile (TMA, rows past the batch zero)
 //   warp 1     issues the MMAs (one thread) and owns the tensor memory
 //   warps 2-5  build the weight operand: the tile's 128 gathered rows, 64
-//              elements per stage, with 128-bit loads (8 threads per row, so
-//              a warp instruction reads four whole 128-byte row pieces) stored
-//              in the swizzled layout; then the epilogue
+//              elements per stage, 8 threads per 128-byte row piece (16-bit
+//              rows: asynchronous copies straight into the swizzled layout;
+//              Q4_0: loads, decode, stores); then the epilogue
 template <int DT, int ACT, int N, int NS>
 __global__ void __launch_bounds__(kUmmaThreads, 2)
     k_umma_up(const __grid_constant__ CUtensorMap tm_x, UmmaParams p) {
@@ -439,6 +445,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       for (int i = 0; i < nst; ++i) {
         const int s = i % NS;
         if (!mbar_wait(&full[s], (i / NS) & 1)) break;
+        if constexpr (!Q4) fence_proxy_async_smem();  // the builders' async copies
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + (size_t)s * STAGE);
         const uint32_t sb = sa + NMAT * ABYTES;
@@ -524,8 +531,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       }
     } else {
       // 16-bit rows: thread m takes chunk c = m % 8 (16 bytes) of rows
-      // 8 (m / 8) + j, j = 0..7, i.e. row j of 8-row group m / 8
-      constexpr int P = umma_ahead16<NMAT>();
+      // 8 (m / 8) + j, j = 0..7, i.e. row j of 8-row group m / 8, and copies
+      // its eight pieces of each stage straight into the swizzled layout
+      // (cp.async, no registers or L1 on the way): up to NS stages in flight
       const int c = m & 7, g = m >> 3;
       const uint8_t* rowp[NMAT][8];
 #pragma unroll
@@ -534,7 +542,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
         rowp[0][j] = p.wa + off;
         if constexpr (NMAT == 2) rowp[NMAT - 1][j] = p.wa2 + off;
       }
-      const uint64_t pol = policy_evict_first();
       // prefetch: thread m asks for row m's 128-byte piece of each stage
       const uint8_t* pfrow[NMAT];
       {
@@ -542,45 +549,29 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
         pfrow[0] = p.wa + off;
         if constexpr (NMAT == 2) pfrow[NMAT - 1] = p.wa2 + off;
       }
-      uint4 raw[P][NMAT][8];
-      auto issue = [&](int i, uint4 (&r)[NMAT][8]) {
+      for (int j = 0; j < kPfAhead && j < nst; ++j)
+#pragma unroll
+        for (int mm = 0; mm < NMAT; ++mm) prefetch_line(pfrow[mm] + 128 * j);
+      const uint32_t gb = smem_u32(smem + g * 1024);
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % NS;
+        if (i + kPfAhead < nst)
+#pragma unroll
+          for (int mm = 0; mm < NMAT; ++mm) prefetch_line(pfrow[mm] + 128 * (i + kPfAhead));
+        if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        const uint32_t st = gb + (uint32_t)(s * STAGE);
 #pragma unroll
         for (int mm = 0; mm < NMAT; ++mm)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) r[mm][j] = ldg_stream_hint(rowp[mm][j] + 128 * i, pol);
-      };
-#pragma unroll
-      for (int j = 0; j < P; ++j)
-        if (j < nst) issue(j, raw[j]);
-      for (int j = P; j < kPfAhead && j < nst; ++j)
-#pragma unroll
-        for (int mm = 0; mm < NMAT; ++mm) prefetch_line(pfrow[mm] + 128 * j);
-      uint8_t* gbase = smem + g * 1024;
-      for (int i0 = 0; i0 < nst && ok; i0 += P) {
-#pragma unroll
-        for (int q = 0; q < P; ++q) {
-          const int i = i0 + q;
-          if (i < nst && ok) {
-            const int s = i % NS;
-            if (i + kPfAhead < nst)
-#pragma unroll
-              for (int mm = 0; mm < NMAT; ++mm) prefetch_line(pfrow[mm] + 128 * (i + kPfAhead));
-            if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
-            if (ok) {
-              uint8_t* st = gbase + (size_t)s * STAGE;
-#pragma unroll
-              for (int mm = 0; mm < NMAT; ++mm)
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                  *reinterpret_cast<uint4*>(st + mm * ABYTES + j * 128 + ((c ^ j) << 4)) =
-                      raw[q][mm][j];
-              fence_proxy_async_smem();
-              mbar_arrive(&full[s]);
-              if (i + P < nst) issue(i + P, raw[q]);
-            }
-          }
-        }
+          for (int j = 0; j < 8; ++j)
+            cp_async16(st + (uint32_t)(mm * ABYTES + j * 128 + ((c ^ j) << 4)),
+                       rowp[mm][j] + 128 * i);
+        cp_async_arrive_noinc(&full[s]);
       }
+      cp_async_wait_all();
     }
     // epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (neurons)
     const int quad = warp & 3;
@@ -677,9 +668,10 @@ __global__ void __launch_bounds__(256) k_umma_up_finish(UmmaParams p) {
 //   warp 0     copies the stage's H tiles, hi and lo (TMA)
 //   warp 1     issues the MMAs and owns the tensor memory
 //   warps 2-5  build the weight operand: 64 neurons x 128 columns per stage,
-//              each neuron's 256-byte row segment read by 16 threads, stored
-//              as one 128-byte row in each of the two column atoms (MN-major,
-//              swizzled); then the epilogue
+//              each neuron's 256-byte row segment taken by 16 threads (16-bit:
+//              asynchronous copies), stored as one 128-byte row in each of
+//              the two column atoms (MN-major, swizzled); then the epilogue.
+//              Q4_0: loads and decode in registers, two threads per neuron
 //   warp 6     reads the neuron ids of the stages ahead and asks the L2 for
 //              their row segments, at most kPfAhead stages ahead of the MMAs
 //              (which publish their progress in shared memory); the ids it
@@ -744,6 +736,7 @@ __global__ void __launch_bounds__(kUmmaDownThreads, 2)
         const int s = i % NS;
         if (!mbar_wait(&full[s], (i / NS) & 1)) break;
         *reinterpret_cast<volatile int*>(&prog) = i;
+        if constexpr (!Q4) fence_proxy_async_smem();  // the builders' async copies
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + (size_t)s * STAGE);
         const uint32_t sh = sa + ABYTES, sl = sh + BBYTES;
@@ -804,7 +797,7 @@ __global__ void __launch_bounds__(kUmmaDownThreads, 2)
         if (id < 0 || id >= p.F) id = -1;  // flagged by the up kernel; zero row
         return id < 0 ? nullptr : p.wd + (size_t)id * p.rb + coff;
       };
-      constexpr int QA = q4_ahead<1>();
+      constexpr int QA = kQ4DownAhead;
       uint32_t raw[QA][9];
       bool live[QA];
 #pragma unroll
@@ -846,11 +839,11 @@ __global__ void __launch_bounds__(kUmmaDownThreads, 2)
       }
     } else {
       // 16-bit rows: thread m takes column chunk c = m % 16 (8 columns) of
-      // neurons 8 (m / 16) + j, j = 0..7 of the stage
-      constexpr int P = 2;
+      // neurons 8 (m / 16) + j, j = 0..7 of the stage, copied straight into
+      // the swizzled layout (cp.async); the next stage's ids are read while
+      // this stage's copies are in flight
       const int c = m & 15, g = m >> 4;
       const uint8_t* cbase = p.wd + (size_t)(col0 + 8 * c) * 2;
-      const uint64_t pol = policy_evict_first();
       auto ids_of = [&](int i, int (&id)[8]) {
         const int kp = (st0 + i) * kUmmaK + 8 * g;
         if (kp + 8 <= K) {
@@ -865,38 +858,24 @@ __global__ void __launch_bounds__(kUmmaDownThreads, 2)
 #pragma unroll
         for (int j = 0; j < 8; ++j) id[j] = (id[j] < 0 || id[j] >= p.F) ? 0 : id[j];
       };
-      uint4 raw[P][8];
       int idn[8];
-      auto issue = [&](int i, uint4 (&r)[8]) {  // ids of stage i are in idn
-#pragma unroll
-        for (int j = 0; j < 8; ++j) r[j] = ldg_stream_hint(cbase + (size_t)idn[j] * p.rb, pol);
-        if (i + 1 < nst) ids_of(i + 1, idn);
-      };
       if (nst > 0) ids_of(0, idn);
-#pragma unroll
-      for (int j = 0; j < P; ++j)
-        if (j < nst) issue(j, raw[j]);
-      uint8_t* gbase = smem + (c >> 3) * (ABYTES / 2) + g * 1024;
       const int cc = c & 7;
-      for (int i0 = 0; i0 < nst && ok; i0 += P) {
-#pragma unroll
-        for (int q = 0; q < P; ++q) {
-          const int i = i0 + q;
-          if (i < nst && ok) {
-            const int s = i % NS;
-            if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
-            if (ok) {
-              uint8_t* st = gbase + (size_t)s * STAGE;
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<uint4*>(st + j * 128 + ((cc ^ j) << 4)) = raw[q][j];
-              fence_proxy_async_smem();
-              mbar_arrive(&full[s]);
-              if (i + P < nst) issue(i + P, raw[q]);
-            }
-          }
+      const uint32_t gb = smem_u32(smem + (c >> 3) * (ABYTES / 2) + g * 1024);
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % NS;
+        if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) {
+          ok = false;
+          break;
         }
+        const uint32_t st = gb + (uint32_t)(s * STAGE);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          cp_async16(st + (uint32_t)(j * 128 + ((cc ^ j) << 4)), cbase + (size_t)idn[j] * p.rb);
+        cp_async_arrive_noinc(&full[s]);
+        if (i + 1 < nst) ids_of(i + 1, idn);
       }
+      cp_async_wait_all();
     }
     const int quad = warp & 3;
     const int col = col0 + quad * 32 + lane;  // output column of this lane
@@ -940,8 +919,8 @@ __global__ void __launch_bounds__(kUmmaDownThreads, 2)
 //     k_pred1_finish sums the slices in order and applies b1 and the ReLU.
 //   warp 0     copies the stage's activation tiles (TMA): a hi and lo, or x
 //   warp 1     issues the MMAs and owns the tensor memory
-//   warps 2-5  load the stage's weight rows (8 threads per 128-byte row piece)
-//              into the swizzled layout; then the epilogue
+//   warps 2-5  copy the stage's weight rows (8 threads per 128-byte row
+//              piece, cp.async) into the swizzled layout; then the epilogue
 struct UmmaPredParams {
   const uint8_t* w;        // [nrows x len] 16-bit rows (W2 or W1)
   const float* bias;       // b2 (layer 2)
@@ -1006,6 +985,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       for (int i = 0; i < nst; ++i) {
         const int s = i % NS;
         if (!mbar_wait(&full[s], (i / NS) & 1)) break;
+        fence_proxy_async_smem();  // the builders' async copies
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + (size_t)s * STAGE);
         const uint32_t sh = sa + ABYTES, sl = sh + BBYTES;
@@ -1021,55 +1001,41 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
     }
     __syncwarp();
   } else {
+    // thread m copies chunk c = m % 8 of rows 8 (m / 8) + j of each stage
+    // straight into the swizzled layout (cp.async; rows past the matrix
+    // are zero-filled)
     const int m = t - 64;
     const int c = m & 7, g = m >> 3;
     const size_t rb = (size_t)p.len * 2;
     const uint8_t* rowp[8];
-    bool live[8];
+    uint32_t nbytes[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int row = row0 + 8 * g + j;
-      live[j] = row < p.nrows;
-      rowp[j] = p.w + (size_t)(live[j] ? row : 0) * rb + (size_t)st0 * 128 + (size_t)c * 16;
+      nbytes[j] = row < p.nrows ? 16u : 0u;
+      rowp[j] = p.w + (size_t)(row < p.nrows ? row : 0) * rb + (size_t)st0 * 128 + (size_t)c * 16;
     }
-    const uint64_t pol = policy_evict_first();
-    constexpr int P = 2;
-    uint4 raw[P][8];
-    auto issue = [&](int i, uint4 (&rr)[8]) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        rr[j] = live[j] ? ldg_stream_hint(rowp[j] + 128 * i, pol) : make_uint4(0, 0, 0, 0);
-    };
-#pragma unroll
-    for (int j = 0; j < P; ++j)
-      if (j < nst) issue(j, raw[j]);
     // prefetch: thread m asks for row m's 128-byte piece of stage i + kPfAhead
     const bool plive = row0 + m < p.nrows;
     const uint8_t* prow = p.w + (size_t)(plive ? row0 + m : 0) * rb + (size_t)st0 * 128;
-    for (int j = P; j < kPfAhead && j < nst; ++j)
+    for (int j = 0; j < kPfAhead && j < nst; ++j)
       if (plive) prefetch_line(prow + 128 * j);
     bool ok = true;
-    uint8_t* gbase = smem + g * 1024;
-    for (int i0 = 0; i0 < nst && ok; i0 += P) {
-#pragma unroll
-      for (int q = 0; q < P; ++q) {
-        const int i = i0 + q;
-        if (i < nst && ok) {
-          const int s = i % NS;
-          if (plive && i + kPfAhead < nst) prefetch_line(prow + 128 * (i + kPfAhead));
-          if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) ok = false;
-          if (ok) {
-            uint8_t* st = gbase + (size_t)s * STAGE;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4*>(st + j * 128 + ((c ^ j) << 4)) = raw[q][j];
-            fence_proxy_async_smem();
-            mbar_arrive(&full[s]);
-            if (i + P < nst) issue(i + P, raw[q]);
-          }
-        }
+    const uint32_t gb = smem_u32(smem + g * 1024);
+    for (int i = 0; i < nst; ++i) {
+      const int s = i % NS;
+      if (plive && i + kPfAhead < nst) prefetch_line(prow + 128 * (i + kPfAhead));
+      if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) {
+        ok = false;
+        break;
       }
+      const uint32_t st = gb + (uint32_t)(s * STAGE);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        cp_async16_fill(st + (uint32_t)(j * 128 + ((c ^ j) << 4)), rowp[j] + 128 * i, nbytes[j]);
+      cp_async_arrive_noinc(&full[s]);
     }
+    cp_async_wait_all();
     // epilogue: lane = row 32 (w % 4) + lane of the tile
     const int quad = warp & 3;
     const int n = row0 + quad * 32 + lane;
