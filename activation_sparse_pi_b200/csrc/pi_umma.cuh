@@ -258,29 +258,35 @@ __device__ __forceinline__ float from16(uint16_t u) {
   else return __uint_as_float((uint32_t)u << 16);
 }
 
-// L2 prefetch of the line holding p, kept in the L2 until used: the operand
-// builders ask for the weight pieces of stage i + kPfAhead while they work on
-// stage i, so the copies and loads of a stage find their lines in the L2.
-// (Measured on the batched kernels: dropping it costs about 30%; longer
-// distances, bursts of a row's pieces and plain eviction priority gain
-// nothing.)
+// L2 prefetch of the line holding p: the operand builders ask for the
+// weight pieces of stage i + kPfAhead while they work on stage i, so the
+// copies and loads of a stage find their lines in the L2.  (Measured on the
+// batched kernels: dropping it costs about 30%; longer distances, bursts of
+// a row's pieces and evict-last priority gain nothing.)
 constexpr int kPfAhead = 8;
 __device__ __forceinline__ void prefetch_line(const void* p) {
-  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // 16-byte asynchronous copy global -> shared that bypasses the L1 (so the
 // bytes in flight are bounded by the pipeline's stage buffers, not by the L1
-// left over after the shared-memory carve-out), and the arrive on an
-// mbarrier once all of this thread's earlier copies have landed (.noinc: the
-// barrier's expected count includes these arrivals).  The consumer fences
-// the async proxy after its wait, before the tensor cores read the stage.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// left over after the shared-memory carve-out), with an L2 policy (the
+// builders pass evict-first: each row piece is read once, and without the
+// hint the consumed lines crowded out prefetched ones, 1.46x the bytes from
+// DRAM on the 13B up projection), and the arrive on an mbarrier once all of
+// this thread's earlier copies have landed (.noinc: the barrier's expected
+// count includes these arrivals).  The consumer fences the async proxy
+// after its wait, before the tensor cores read the stage.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "l"(pol)
+               : "memory");
 }
 // Same, reading src_bytes (0 or 16) and filling the rest of the 16 with zeros.
-__device__ __forceinline__ void cp_async16_fill(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+__device__ __forceinline__ void cp_async16_fill(uint32_t dst, const void* src, uint32_t src_bytes,
+                                                uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst),
+               "l"(src), "r"(src_bytes), "l"(pol)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
@@ -553,6 +559,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
 #pragma unroll
         for (int mm = 0; mm < NMAT; ++mm) prefetch_line(pfrow[mm] + 128 * j);
       const uint32_t gb = smem_u32(smem + g * 1024);
+      const uint64_t pol = policy_evict_first();  // a row piece is read once
       for (int i = 0; i < nst; ++i) {
         const int s = i % NS;
         if (i + kPfAhead < nst)
@@ -568,7 +575,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             cp_async16(st + (uint32_t)(mm * ABYTES + j * 128 + ((c ^ j) << 4)),
-                       rowp[mm][j] + 128 * i);
+                       rowp[mm][j] + 128 * i, pol);
         cp_async_arrive_noinc(&full[s]);
       }
       cp_async_wait_all();
@@ -862,6 +869,7 @@ __global__ void __launch_bounds__(kUmmaDownThreads, 2)
       if (nst > 0) ids_of(0, idn);
       const int cc = c & 7;
       const uint32_t gb = smem_u32(smem + (c >> 3) * (ABYTES / 2) + g * 1024);
+      const uint64_t pol = policy_evict_first();
       for (int i = 0; i < nst; ++i) {
         const int s = i % NS;
         if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) {
@@ -871,7 +879,7 @@ __global__ void __launch_bounds__(kUmmaDownThreads, 2)
         const uint32_t st = gb + (uint32_t)(s * STAGE);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          cp_async16(st + (uint32_t)(j * 128 + ((cc ^ j) << 4)), cbase + (size_t)idn[j] * p.rb);
+          cp_async16(st + (uint32_t)(j * 128 + ((cc ^ j) << 4)), cbase + (size_t)idn[j] * p.rb, pol);
         cp_async_arrive_noinc(&full[s]);
         if (i + 1 < nst) ids_of(i + 1, idn);
       }
@@ -1022,6 +1030,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       if (plive) prefetch_line(prow + 128 * j);
     bool ok = true;
     const uint32_t gb = smem_u32(smem + g * 1024);
+    const uint64_t pol = policy_evict_first();
     for (int i = 0; i < nst; ++i) {
       const int s = i % NS;
       if (plive && i + kPfAhead < nst) prefetch_line(prow + 128 * (i + kPfAhead));
@@ -1032,7 +1041,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       const uint32_t st = gb + (uint32_t)(s * STAGE);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        cp_async16_fill(st + (uint32_t)(j * 128 + ((c ^ j) << 4)), rowp[j] + 128 * i, nbytes[j]);
+        cp_async16_fill(st + (uint32_t)(j * 128 + ((c ^ j) << 4)), rowp[j] + 128 * i, nbytes[j],
+                        pol);
       cp_async_arrive_noinc(&full[s]);
     }
     cp_async_wait_all();

@@ -492,6 +492,7 @@ def run_ours(args, rank, world, local):
     if args.layers:
         cfg = dataclasses.replace(cfg, n_layers=min(args.layers, cfg.n_layers))
     B, T, NL, d, F = args.batch, cfg.n_tokens, cfg.n_layers, cfg.d_model, cfg.d_ff
+    T = max(B, T // B * B)  # whole batches: a batch that does not divide the tokens drops the rest
     peak, peak_kind = measured_hbm()
 
     def barrier():
@@ -651,7 +652,7 @@ def run_ours(args, rank, world, local):
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.wdtype,
-            "data": "synthetic", "config": workload_config(cfg, args.mode, B),
+            "data": "synthetic", "config": workload_config(cfg, args.mode, B, tokens=T),
             "roofline": roofline, "stack_roofline": stack_roof,
             "gpu_launches": int(launches_per_step * args.steps),
             "clocks": clocks,
