@@ -56,7 +56,7 @@ SAMPLE_LAYERS = 4         # layers of the oracle sample (both arms)
 # launch's algorithmic bytes, with the hash of the sources that define the
 # kernel (k_ffn_ldg: pi_common.cuh, pi_predict.cuh, pi_ffn.cuh) when it was
 # taken; a changed kernel invalidates it.
-TRAFFIC = {"ratio": 1.070, "src_sha": "24dcaa110b6d3731", "config": "falcon-40b",
+TRAFFIC = {"ratio": 1.074, "src_sha": "f8e9a7df2cab9f58", "config": "falcon-40b",
            "files": ("pi_common.cuh", "pi_predict.cuh", "pi_ffn.cuh"),
            "profile": "profiles/k_ffn_ldg_falcon40b_2layer.md"}
 
