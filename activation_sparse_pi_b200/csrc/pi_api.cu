@@ -387,22 +387,23 @@ cudaError_t pred2_cpl(const pi_predictor* P, const float* a, uint32_t* mask, flo
 
 // batches of 8+ with 16-bit rows: tensor-core tiles of 16 rows x 8 tokens
 template <int MODE, int WDT, int ACT, int NT>
-cudaError_t launch_rows_mma_nt(const RowsParams& p, int tiles, cudaStream_t st) {
+cudaError_t launch_rows_mma_nt(const RowsParams& p, int tiles, int Y, cudaStream_t st) {
   constexpr int NUP = (MODE == kModeUp && ACT == 1) ? 2 : 1;
   const size_t smem = (size_t)kMmaWarps * NUP * NT * 4 * 32 * sizeof(float);
-  return launch(k_rows_mma<MODE, WDT, ACT, NT>, dim3(tiles), dim3(32 * kMmaWarps), smem, st, p);
+  return launch(k_rows_mma<MODE, WDT, ACT, NT>, dim3(tiles, Y), dim3(32 * kMmaWarps), smem, st, p);
 }
 
 // one CTA per tile of 16 rows (the upper bound nrows_work; CTAs past the
-// device-side row count return at once)
+// device-side row count return at once) and slice of the contraction (Y > 1:
+// predictor layer 1 only, raw sums to p.part)
 template <int MODE, int WDT, int ACT>
-cudaError_t launch_rows_mma(const RowsParams& p, int nrows_work, cudaStream_t st) {
+cudaError_t launch_rows_mma(const RowsParams& p, int nrows_work, cudaStream_t st, int Y = 1) {
   const int tiles = std::max(1, (nrows_work + 15) / 16);
   const int nt = (p.B + 7) / 8;
-  if (nt <= 1) return launch_rows_mma_nt<MODE, WDT, ACT, 1>(p, tiles, st);
-  if (nt <= 2) return launch_rows_mma_nt<MODE, WDT, ACT, 2>(p, tiles, st);
-  if (nt <= 4) return launch_rows_mma_nt<MODE, WDT, ACT, 4>(p, tiles, st);
-  return launch_rows_mma_nt<MODE, WDT, ACT, 8>(p, tiles, st);
+  if (nt <= 1) return launch_rows_mma_nt<MODE, WDT, ACT, 1>(p, tiles, Y, st);
+  if (nt <= 2) return launch_rows_mma_nt<MODE, WDT, ACT, 2>(p, tiles, Y, st);
+  if (nt <= 4) return launch_rows_mma_nt<MODE, WDT, ACT, 4>(p, tiles, Y, st);
+  return launch_rows_mma_nt<MODE, WDT, ACT, 8>(p, tiles, Y, st);
 }
 
 template <int DT, int MODE, int BB>
@@ -556,7 +557,7 @@ cudaError_t umma_predict(const pi_predictor* P, int B, const uint16_t* x, uint16
   cudaError_t e = umma_pred_n<true, DT>(N, r, S, tx, tx, p1, st);
   if (e != cudaSuccess) return e;
   e = launch(k_pred1_finish<DT>, dim3((B * r + 255) / 256), dim3(256), 0, st, (const float*)part,
-             S, B, r, P->b1, ah, al);
+             S, B, r, P->b1, ah, al, (float*)nullptr);
   if (e != cudaSuccess) return e;
   UmmaPredParams p2{};
   p2.w = static_cast<const uint8_t*>(P->w2);
@@ -620,7 +621,21 @@ int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const fl
     p.nrows = P->rank;
     p.len = d;
     p.B = B;
-    PI_CUDA((rows_bb<DT, kModePred1>(p, P->rank, st)));
+    // batch 8-15: the r/16 row tiles leave most SMs idle, so the contraction
+    // is also split (about two CTAs per SM), the raw sums go to the scratch
+    // and k_pred1_finish adds them in slice order with b1 and the ReLU
+    const int tiles = P->rank / 16;
+    int Y = std::min(8, std::max(1, 2 * num_sms() / std::max(1, tiles)));
+    Y = (int)std::min<size_t>((size_t)Y, part_bytes / ((size_t)B * P->rank * 4));
+    if (B >= 8 && part && Y > 1) {
+      p.part = part;
+      PI_CUDA((launch_rows_mma<kModePred1, DT, 0>(p, P->rank, st, Y)));
+      PI_CUDA((launch(k_pred1_finish<DT>, dim3((B * P->rank + 255) / 256), dim3(256), 0, st,
+                      (const float*)part, Y, B, P->rank, P->b1, (uint16_t*)nullptr,
+                      (uint16_t*)nullptr, a)));
+    } else {
+      PI_CUDA((rows_bb<DT, kModePred1>(p, P->rank, st)));
+    }
   }
   if (pred2_fused_ok(B, P->rank)) {
     if (B == 1) PI_CUDA((pred2_cpl<DT, 1>(P, a, mask, logits, st)));
@@ -638,9 +653,20 @@ int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const fl
     p.F = P->d_ff;
     p.r = P->rank;
     p.B = B;
-    const dim3 grid(P->d_ff / 32, (B + 7) / 8);
-    if (P->rank <= 1024) PI_CUDA((launch(k_pred2_words<DT, 4>, grid, dim3(256), 0, st, p)));
-    else PI_CUDA((launch(k_pred2_words<DT, 8>, grid, dim3(256), 0, st, p)));
+    // a CTA per mask word, or per half word when that fills the two CTAs per
+    // SM better (the last wave of whole words can leave most SMs idle)
+    const int slots = 2 * num_sms(), w32 = P->d_ff / 32, w16 = P->d_ff / 16;
+    const double e32 = (double)w32 / (slots * ((w32 + slots - 1) / slots));
+    const double e16 = (double)w16 / (slots * ((w16 + slots - 1) / slots));
+    const bool half = e16 > e32 + 0.05;
+    const dim3 grid(half ? w16 : w32, (B + 7) / 8);
+    if (P->rank <= 1024) {
+      if (half) PI_CUDA((launch(k_pred2_words<DT, 4, 16>, grid, dim3(256), 0, st, p)));
+      else PI_CUDA((launch(k_pred2_words<DT, 4, 32>, grid, dim3(256), 0, st, p)));
+    } else {
+      if (half) PI_CUDA((launch(k_pred2_words<DT, 8, 16>, grid, dim3(256), 0, st, p)));
+      else PI_CUDA((launch(k_pred2_words<DT, 8, 32>, grid, dim3(256), 0, st, p)));
+    }
   }
   return PI_OK;
 }

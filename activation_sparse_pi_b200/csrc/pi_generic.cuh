@@ -46,6 +46,8 @@ struct RowsParams {
   float* out;              // a [B x r] | logits [B x F] (nullable) | h [K x B]
   uint16_t* out_hi;        // pred1 on tensor cores (optional): a as 16-bit hi + lo
   uint16_t* out_lo;        //   parts [B x r], the operand of the tcgen05 layer 2
+  float* part;             // pred1 split over the contraction (gridDim.y > 1):
+                           //   [gridDim.y x B x r] raw sums, finished by k_pred1_finish
   uint32_t* mask;          // [B x F/32] (pred2)
   float threshold;
   int nrows;               // r | F | F (bound on K)
@@ -222,19 +224,20 @@ struct Pred2WordsParams {
   int F, r, B;
 };
 
-template <int DT, int NQ>
+template <int DT, int NQ, int RU>
 __global__ void __launch_bounds__(256) k_pred2_words(Pred2WordsParams p) {
+  static_assert(RU == 32 || RU == 16, "a CTA takes a mask word or half of one");
   constexpr int RS = 8 / NQ;          // row streams
-  constexpr int ROWS = 32 / RS;       // rows per warp
+  constexpr int ROWS = RU / RS;       // rows per warp
   constexpr int U = 4;                // rows whose chunks are in flight together
-  __shared__ float part[32][NQ][8];
+  __shared__ float part[RU][NQ][8];
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int q = warp % NQ, rs = warp / NQ;
-  const int word = blockIdx.x, b0 = blockIdx.y * 8;
+  const int unit = blockIdx.x, b0 = blockIdx.y * 8;
   const size_t rb = (size_t)p.r * 2;
-  const uint8_t* slab = p.w2 + (size_t)word * 32 * rb;
-  if (t == 0) {  // the word's 32 rows, contiguous: stream them into the L2 now
-    const size_t bytes = 32 * rb;
+  const uint8_t* slab = p.w2 + (size_t)unit * RU * rb;
+  if (t == 0) {  // the unit's rows, contiguous: stream them into the L2 now
+    const size_t bytes = RU * rb;
     for (size_t o = 0; o < bytes; o += 32768)
       prefetch_l2(slab + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768));
   }
@@ -281,16 +284,26 @@ __global__ void __launch_bounds__(256) k_pred2_words(Pred2WordsParams p) {
     }
   }
   __syncthreads();
-  // warp b: token b0 + b, lane = row of the word
-  const int b = warp, n = word * 32 + lane;
+  // warp b: token b0 + b, lane = row of the unit.  A half-word unit (RU 16)
+  // writes its 16 bits as one half of the little-endian mask word, so two
+  // CTAs fill a word without atomics.
+  const int b = warp, n = unit * RU + lane;
   if (b0 + b < p.B) {  // warp-uniform
     float sv = 0.f;
+    if (lane < RU) {
 #pragma unroll
-    for (int g = 0; g < NQ; ++g) sv += part[lane][g][b];
-    sv += p.b2[n];
-    if (p.logits) p.logits[(size_t)(b0 + b) * p.F + n] = sv;
-    const uint32_t bits = __ballot_sync(0xffffffffu, sv > p.threshold);
-    if (lane == 0) p.mask[(size_t)(b0 + b) * (p.F / 32) + word] = bits;
+      for (int g = 0; g < NQ; ++g) sv += part[lane][g][b];
+      sv += p.b2[n];
+      if (p.logits) p.logits[(size_t)(b0 + b) * p.F + n] = sv;
+    }
+    const uint32_t bits = __ballot_sync(0xffffffffu, lane < RU && sv > p.threshold);
+    if (lane == 0) {
+      if constexpr (RU == 32)
+        p.mask[(size_t)(b0 + b) * (p.F / 32) + unit] = bits;
+      else
+        reinterpret_cast<uint16_t*>(p.mask)[(size_t)(b0 + b) * (p.F / 16) + unit] =
+            (uint16_t)bits;
+    }
   }
 }
 
@@ -535,9 +548,14 @@ __global__ void __launch_bounds__(32 * kMmaWarps) k_rows_mma(RowsParams p) {
   if (tile * 16 >= nrows) return;  // whole CTA: no barrier is skipped by part of it
   const int B = p.B;
   const int len = p.len;
+  // the contraction in 32-element steps: slice blockIdx.y of gridDim.y (the
+  // predictor's layer 1 has only r/16 tiles), then split among the warps
   const int nsteps = len / 32;
-  const int s_lo = (int)(((long long)nsteps * warp) / kMmaWarps);
-  const int s_hi = (int)(((long long)nsteps * (warp + 1)) / kMmaWarps);
+  const int Y = gridDim.y;
+  const int c_lo = (int)(((long long)nsteps * blockIdx.y) / Y);
+  const int c_n = (int)(((long long)nsteps * (blockIdx.y + 1)) / Y) - c_lo;
+  const int s_lo = c_lo + (int)(((long long)c_n * warp) / kMmaWarps);
+  const int s_hi = c_lo + (int)(((long long)c_n * (warp + 1)) / kMmaWarps);
   const size_t rb = (size_t)len * 2;
   const uint64_t pol = policy_evict_first();
 
@@ -633,7 +651,9 @@ __global__ void __launch_bounds__(32 * kMmaWarps) k_rows_mma(RowsParams p) {
       const int tok = n * 8 + 2 * t + (e & 1);
       if (row < nrows && tok < B) {
         const float bias = p.bias ? p.bias[nid[hlf]] : 0.f;
-        if constexpr (MODE == kModePred1) {
+        if (MODE == kModePred1 && Y > 1) {
+          p.part[((size_t)blockIdx.y * B + tok) * p.nrows + row] = acc[0][n][e];
+        } else if constexpr (MODE == kModePred1) {
           const float a = fmaxf(acc[0][n][e] + bias, 0.f);
           p.out[(size_t)tok * p.nrows + row] = a;
           if (p.out_hi) {

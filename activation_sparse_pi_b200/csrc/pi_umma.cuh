@@ -1102,13 +1102,15 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
 }
 
 // Predictor layer 1 from its split-contraction partials: a = relu(sum over
-// the S slices in order + b1), written as the hi + lo 16-bit parts that layer
-// 2 multiplies.  part [S x B x r].
+// the S slices in order + b1), written as fp32 (aout, for the CUDA-core
+// layer 2) and/or as the hi + lo 16-bit parts that the tensor-core layer 2
+// multiplies (ahi, alo).  part [S x B x r].
 template <int DT>
 __global__ void __launch_bounds__(256) k_pred1_finish(const float* __restrict__ part, int S, int B,
                                                       int r, const float* __restrict__ b1,
                                                       uint16_t* __restrict__ ahi,
-                                                      uint16_t* __restrict__ alo) {
+                                                      uint16_t* __restrict__ alo,
+                                                      float* __restrict__ aout) {
   pdl_wait();
   pdl_trigger();
   const int e = blockIdx.x * 256 + threadIdx.x;
@@ -1117,9 +1119,12 @@ __global__ void __launch_bounds__(256) k_pred1_finish(const float* __restrict__ 
   for (int y = 1; y < S; ++y) z += part[(size_t)y * B * r + e];
   if (b1) z += b1[e % r];
   const float a = fmaxf(z, 0.f);
-  const uint16_t hi = to16<DT>(a);
-  ahi[e] = hi;
-  alo[e] = to16<DT>(a - from16<DT>(hi));
+  if (aout) aout[e] = a;
+  if (ahi) {
+    const uint16_t hi = to16<DT>(a);
+    ahi[e] = hi;
+    alo[e] = to16<DT>(a - from16<DT>(hi));
+  }
 }
 
 }  // namespace pi
