@@ -234,10 +234,13 @@ int32_t check_ws(void* ws, size_t have, size_t need) {
 }
 
 // ------------------------------------------------- tensor-core batched path
-// Batches of at least kUmmaMinBatch tokens with 16-bit weights run the
-// gathered up and down projections as tcgen05 GEMMs (pi_umma.cuh); their
+// Batches of at least kUmmaMinBatch tokens that the fused batch-1/2/4
+// kernels do not take run the gathered up and down projections as tcgen05
+// GEMMs (pi_umma.cuh), N = the batch rounded up to 16: the rows are read
+// once either way, and the tensor cores leave the CUDA cores' FMA issue
+// (half the issue slots of the batch-5 row kernels) out of the path.  Their
 // operands are described to the copy engine by tensor maps built here.
-constexpr int kUmmaMinBatch = 8;
+constexpr int kUmmaMinBatch = 3;
 
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
