@@ -44,8 +44,6 @@ struct RowsParams {
   const int32_t* idx;      // gathered rows (up)
   const int32_t* count;
   float* out;              // a [B x r] | logits [B x F] (nullable) | h [K x B]
-  uint16_t* out_hi;        // pred1 on tensor cores (optional): a as 16-bit hi + lo
-  uint16_t* out_lo;        //   parts [B x r], the operand of the tcgen05 layer 2
   float* part;             // pred1 split over the contraction (gridDim.y > 1):
                            //   [gridDim.y x B x r] raw sums, finished by k_pred1_finish
   uint32_t* mask;          // [B x F/32] (pred2)
@@ -656,13 +654,6 @@ __global__ void __launch_bounds__(32 * kMmaWarps) k_rows_mma(RowsParams p) {
         } else if constexpr (MODE == kModePred1) {
           const float a = fmaxf(acc[0][n][e] + bias, 0.f);
           p.out[(size_t)tok * p.nrows + row] = a;
-          if (p.out_hi) {
-            const uint16_t hi = round16<WDT>(a);
-            const float fh = WDT == 0 ? __half2float(__ushort_as_half(hi))
-                                      : __uint_as_float((uint32_t)hi << 16);
-            p.out_hi[(size_t)tok * p.nrows + row] = hi;
-            p.out_lo[(size_t)tok * p.nrows + row] = round16<WDT>(a - fh);
-          }
         } else {
           float h = fmaxf(acc[0][n][e] + (ok[hlf] ? bias : 0.f), 0.f);
           if constexpr (ACT == 1) h *= acc[NUP - 1][n][e];
