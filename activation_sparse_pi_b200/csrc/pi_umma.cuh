@@ -260,10 +260,14 @@ __device__ __forceinline__ float from16(uint16_t u) {
 
 // L2 prefetch of the line holding p: the operand builders ask for the
 // weight pieces of stage i + kPfAhead while they work on stage i, so the
-// copies and loads of a stage find their lines in the L2.  (Measured on the
-// batched kernels: dropping it costs about 30%; longer distances, bursts of
-// a row's pieces and evict-last priority gain nothing.)
-constexpr int kPfAhead = 8;
+// copies and loads of a stage find their lines in the L2.  Measured on the
+// batched kernels: dropping it costs 10-30%; for the 16-bit builders, whose
+// asynchronous copies are already up to six stages ahead, 4 stages beat 8
+// by 3-7% (12 and 16 are slower); the Q4_0 builders, which load a
+// super-stage at a time into registers, want 8 (two super-stages).
+// Bursts of a row's pieces and evict-last priority gain nothing.
+constexpr int kPfAhead = 4;
+constexpr int kPfAheadQ4 = 8;
 __device__ __forceinline__ void prefetch_line(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
@@ -485,7 +489,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       rowp[0] = p.wa + roff;
       if constexpr (NMAT == 2) rowp[NMAT - 1] = p.wa2 + roff;
       const int nss = nst / 4;  // super-stages
-      constexpr int SSA = kPfAhead / 4;
+      constexpr int SSA = kPfAheadQ4 / 4;
       auto pf_ss = [&](int ss) {
 #pragma unroll
         for (int mm = 0; mm < NMAT; ++mm) {
@@ -680,7 +684,7 @@ __global__ void __launch_bounds__(256) k_umma_up_finish(UmmaParams p) {
 //              the two column atoms (MN-major, swizzled); then the epilogue.
 //              Q4_0: loads and decode in registers, two threads per neuron
 //   warp 6     reads the neuron ids of the stages ahead and asks the L2 for
-//              their row segments, at most kPfAhead stages ahead of the MMAs
+//              their row segments, at most kPfAhead (Q4_0: kPfAheadQ4) stages ahead of the MMAs
 //              (which publish their progress in shared memory); the ids it
 //              reads are then in the L1 for the builders
 template <int DT, int N, int NS>
@@ -766,7 +770,8 @@ __global__ void __launch_bounds__(kUmmaDownThreads, 2)
     const int span = Q4 ? 71 : 255;  // last byte of a neuron's segment
     for (int j = 0; j < nst; ++j) {
       uint32_t it = 0;
-      while (*reinterpret_cast<volatile int*>(&prog) < j - kPfAhead && ++it < kWaitLimitSleep)
+      while (*reinterpret_cast<volatile int*>(&prog) < j - (Q4 ? kPfAheadQ4 : kPfAhead) &&
+             ++it < kWaitLimitSleep)
         __nanosleep(128);
       if (it >= kWaitLimitSleep) break;  // only a hint: stop prefetching
       const int kp = (st0 + j) * kUmmaK + 2 * lane;
