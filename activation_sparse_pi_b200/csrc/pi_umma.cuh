@@ -9,12 +9,14 @@
 //   down: y[n][c]  = sum_k H[k][n] W_down^T[idx_k][c]
 // Both run here as tcgen05.mma (kind::f16, fp32 accumulation in tensor
 // memory) on operands staged in 128-byte-swizzled shared memory:
-//   - weight rows: four warps gather the listed rows with coalesced 128-bit
-//     loads (eight threads per 128-byte piece of a row) and store them in
-//     the swizzled layout, dequantizing Q4_0 blocks on the way.  (A first
-//     version gathered them with cp.async.bulk.tensor .tile::gather4; at 128
+//   - weight rows: four warps gather the listed rows, eight threads per
+//     128-byte piece of a row.  16-bit pieces go straight into the swizzled
+//     layout with 16-byte cp.async copies (no registers or L1 on the way);
+//     Q4_0 blocks are loaded into registers, dequantized and stored.  Every
+//     builder asks the L2 for its pieces a few stages ahead.  (A first
+//     version gathered rows with cp.async.bulk.tensor .tile::gather4; at 128
 //     bytes per row and four rows per instruction the copy engine delivered
-//     about 1.7 TB/s, a quarter of what plain loads reach.)
+//     about 1.7 TB/s, a quarter of what the copies here reach.)
 //   - tokens (up) and H (down): 2-D tensor tiles copied by the tensor memory
 //     accelerator, rows past the batch filled with zeros by the copy engine.
 // One thread issues the copies, one thread the MMAs; the four builder warps
