@@ -656,13 +656,13 @@ int32_t predict_impl(const pi_predictor* P, int B, const uint16_t* x16, const fl
     p.F = P->d_ff;
     p.r = P->rank;
     p.B = B;
-    // a CTA per mask word, or per half word when that fills the two CTAs per
-    // SM better (the last wave of whole words can leave most SMs idle)
+    // units of a mask word, or of half a word when that spreads them more
+    // evenly over the two CTAs per SM; each CTA loops over its units
     const int slots = 2 * num_sms(), w32 = P->d_ff / 32, w16 = P->d_ff / 16;
     const double e32 = (double)w32 / (slots * ((w32 + slots - 1) / slots));
     const double e16 = (double)w16 / (slots * ((w16 + slots - 1) / slots));
     const bool half = e16 > e32 + 0.05;
-    const dim3 grid(half ? w16 : w32, (B + 7) / 8);
+    const dim3 grid(std::min(half ? w16 : w32, slots), (B + 7) / 8);
     if (P->rank <= 1024) {
       if (half) PI_CUDA((launch(k_pred2_words<DT, 4, 16>, grid, dim3(256), 0, st, p)));
       else PI_CUDA((launch(k_pred2_words<DT, 4, 32>, grid, dim3(256), 0, st, p)));

@@ -224,21 +224,26 @@ struct Pred2WordsParams {
 
 template <int DT, int NQ, int RU>
 __global__ void __launch_bounds__(256) k_pred2_words(Pred2WordsParams p) {
-  static_assert(RU == 32 || RU == 16, "a CTA takes a mask word or half of one");
+  static_assert(RU == 32 || RU == 16, "a unit is a mask word or half of one");
   constexpr int RS = 8 / NQ;          // row streams
   constexpr int ROWS = RU / RS;       // rows per warp
   constexpr int U = 4;                // rows whose chunks are in flight together
   __shared__ float part[RU][NQ][8];
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int q = warp % NQ, rs = warp / NQ;
-  const int unit = blockIdx.x, b0 = blockIdx.y * 8;
+  const int b0 = blockIdx.y * 8;
+  const int nunits = p.F / RU;
   const size_t rb = (size_t)p.r * 2;
-  const uint8_t* slab = p.w2 + (size_t)unit * RU * rb;
-  if (t == 0) {  // the unit's rows, contiguous: stream them into the L2 now
+  // the CTA takes units blockIdx.x, + gridDim.x, ...: the activations a of
+  // its 8 tokens are loaded once and serve every unit (one unit per CTA
+  // re-read as many bytes of a from the L2 as of W2)
+  auto prefetch_unit = [&](int unit) {  // a unit's rows are contiguous
+    const uint8_t* slab = p.w2 + (size_t)unit * RU * rb;
     const size_t bytes = RU * rb;
     for (size_t o = 0; o < bytes; o += 32768)
       prefetch_l2(slab + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768));
-  }
+  };
+  if (t == 0 && blockIdx.x < nunits) prefetch_unit(blockIdx.x);
   pdl_wait();
   pdl_trigger();
   const int nch = p.r / 8;
@@ -255,53 +260,58 @@ __global__ void __launch_bounds__(256) k_pred2_words(Pred2WordsParams p) {
     av[b][0] = lo.x; av[b][1] = lo.y; av[b][2] = lo.z; av[b][3] = lo.w;
     av[b][4] = hi.x; av[b][5] = hi.y; av[b][6] = hi.z; av[b][7] = hi.w;
   }
-  for (int r0 = 0; r0 < ROWS; r0 += U) {
-    uint4 w[U];
+  for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
+    if (t == 0 && unit + (int)gridDim.x < nunits) prefetch_unit(unit + gridDim.x);
+    const uint8_t* slab = p.w2 + (size_t)unit * RU * rb;
+    for (int r0 = 0; r0 < ROWS; r0 += U) {
+      uint4 w[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int row = rs * ROWS + r0 + u;
-      w[u] = mine ? ldg_stream(slab + (size_t)row * rb + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      float v[8];
-      const uint32_t wv[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        float z = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = unpack2<DT>(wv[e]);
-          z = fmaf(f.x, av[b][2 * e], z);
-          z = fmaf(f.y, av[b][2 * e + 1], z);
-        }
-        v[b] = z;
+      for (int u = 0; u < U; ++u) {
+        const int row = rs * ROWS + r0 + u;
+        w[u] = mine ? ldg_stream(slab + (size_t)row * rb + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
       }
-      const float tot = warp_reduce_transposed<8>(v);  // lane holds token lane / 4
-      if ((lane & 3) == 0) part[rs * ROWS + r0 + u][q][lane >> 2] = tot;
-    }
-  }
-  __syncthreads();
-  // warp b: token b0 + b, lane = row of the unit.  A half-word unit (RU 16)
-  // writes its 16 bits as one half of the little-endian mask word, so two
-  // CTAs fill a word without atomics.
-  const int b = warp, n = unit * RU + lane;
-  if (b0 + b < p.B) {  // warp-uniform
-    float sv = 0.f;
-    if (lane < RU) {
 #pragma unroll
-      for (int g = 0; g < NQ; ++g) sv += part[lane][g][b];
-      sv += p.b2[n];
-      if (p.logits) p.logits[(size_t)(b0 + b) * p.F + n] = sv;
+      for (int u = 0; u < U; ++u) {
+        float v[8];
+        const uint32_t wv[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          float z = 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack2<DT>(wv[e]);
+            z = fmaf(f.x, av[b][2 * e], z);
+            z = fmaf(f.y, av[b][2 * e + 1], z);
+          }
+          v[b] = z;
+        }
+        const float tot = warp_reduce_transposed<8>(v);  // lane holds token lane / 4
+        if ((lane & 3) == 0) part[rs * ROWS + r0 + u][q][lane >> 2] = tot;
+      }
     }
-    const uint32_t bits = __ballot_sync(0xffffffffu, lane < RU && sv > p.threshold);
-    if (lane == 0) {
-      if constexpr (RU == 32)
-        p.mask[(size_t)(b0 + b) * (p.F / 32) + unit] = bits;
-      else
-        reinterpret_cast<uint16_t*>(p.mask)[(size_t)(b0 + b) * (p.F / 16) + unit] =
-            (uint16_t)bits;
+    __syncthreads();
+    // warp b: token b0 + b, lane = row of the unit.  A half-word unit (RU 16)
+    // writes its 16 bits as one half of the little-endian mask word, so two
+    // units fill a word without atomics.
+    const int b = warp, n = unit * RU + lane;
+    if (b0 + b < p.B) {  // warp-uniform
+      float sv = 0.f;
+      if (lane < RU) {
+#pragma unroll
+        for (int g = 0; g < NQ; ++g) sv += part[lane][g][b];
+        sv += p.b2[n];
+        if (p.logits) p.logits[(size_t)(b0 + b) * p.F + n] = sv;
+      }
+      const uint32_t bits = __ballot_sync(0xffffffffu, lane < RU && sv > p.threshold);
+      if (lane == 0) {
+        if constexpr (RU == 32)
+          p.mask[(size_t)(b0 + b) * (p.F / 32) + unit] = bits;
+        else
+          reinterpret_cast<uint16_t*>(p.mask)[(size_t)(b0 + b) * (p.F / 16) + unit] =
+              (uint16_t)bits;
+      }
     }
+    __syncthreads();  // part is rewritten by the next unit
   }
 }
 
