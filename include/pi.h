@@ -175,8 +175,9 @@ int32_t pi_compact(const uint32_t* mask_bits, int32_t batch, int32_t d_ff,
  *   y      [batch x d_model] fp32 out (overwritten)
  * The summation order is fixed, so repeated calls give bit-identical y.
  * Passing idx = 0..d_ff-1 and count = d_ff gives the dense FFN.
- * At batch >= 8 (d_model % 128 == 0) the up and down projections run on the
- * tensor cores: products of 16-bit operands accumulate in fp32, the
+ * At batches 3 and 5-64 (and 4 with Q4_0 weights), with d_model % 128 == 0,
+ * the up and down projections run on the tensor cores (batches 1, 2 and 4 use
+ * fused CUDA-core kernels): products of 16-bit operands accumulate in fp32, the
  * activations h enter the down projection as a hi + lo pair of 16-bit values
  * (about 16 significant bits with bf16 weights, 22 with fp16), and Q4_0
  * weights are rounded once to fp16 after dequantization (relative 2^-12).
